@@ -1,0 +1,241 @@
+"""fp64 CPU oracle of the NOSA sparse-decode step.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
+and by ``bench.py``'s CPU-baseline / reference leg, never by the product
+package. It shares no code with the CUDA library; the only thing both sides use
+is the input generator in ``nosa_synth`` (random numbers, no method arithmetic).
+
+``nosa_oracle.c`` holds the arithmetic (see its header for the passages it
+follows); this module loads it with ctypes, keeps the oracle's state in numpy
+arrays, and builds margin-checked test cases (:func:`run_case`).
+
+Parity status: every oracle function is pinned by ``tests/test_oracle_pins.py``
+(library routines, brute force, closed forms, invariants and a hand-worked
+example); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import shutil
+import subprocess
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import numpy as np
+
+import nosa_synth as syn
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nosa_oracle.c")
+_SO = os.path.join(_HERE, "libnosa_oracle.so")
+
+MARGIN = 1e-3  # score margin required at the query-aware cut
+
+
+def compile_oracle(src: str, out: str) -> str:
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", out,
+                           src, "-lm"])
+    return out
+
+
+def build(force: bool = False) -> str:
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        compile_oracle(_SRC, _SO)
+    return _SO
+
+
+class OrcCfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "Hq", "Hkv", "d", "bs", "s", "k_q", "k_e", "n_rows", "max_blocks", "slots",
+                 "offload")] + [("scale", ctypes.c_double)]
+
+
+class OrcState(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("K", "V", "kbar", "len", "prev_sel", "alive", "block_slot", "slot_owner",
+                 "last_used")]
+
+
+_libs = {}
+
+
+def load(path: Optional[str] = None):
+    path = path or build()
+    if path not in _libs:
+        L = ctypes.CDLL(path)
+        vp = ctypes.c_void_p
+        L.orc_topm.argtypes = [ctypes.c_int, vp, vp, ctypes.c_int, vp, vp]
+        L.orc_topm.restype = ctypes.c_int
+        L.orc_init.argtypes = [vp, vp, vp, vp]
+        L.orc_init.restype = ctypes.c_int
+        L.orc_append.argtypes = [vp, vp, vp, vp]
+        L.orc_append.restype = None
+        L.orc_block_scores.argtypes = [vp, vp, vp, vp]
+        L.orc_block_scores.restype = None
+        L.orc_select.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_int]
+        L.orc_select.restype = None
+        L.orc_residency.argtypes = [vp, vp, vp, vp]
+        L.orc_residency.restype = ctypes.c_int
+        L.orc_attend.argtypes = [vp, vp, vp, vp, vp]
+        L.orc_attend.restype = None
+        _libs[path] = L
+    return _libs[path]
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def topm(key: np.ndarray, cand: np.ndarray, m: int, lib=None):
+    """Top-m of key over cand (ties to the lower index): (chosen uint8, gap)."""
+    L = lib or load()
+    key = np.ascontiguousarray(key, np.float64)
+    cand = np.ascontiguousarray(cand, np.uint8)
+    ch = np.zeros(key.size, np.uint8)
+    gap = np.zeros(1, np.float64)
+    L.orc_topm(key.size, _p(key), _p(cand), m, _p(ch), _p(gap))
+    return ch, float(gap[0])
+
+
+class Oracle:
+    """Oracle state for one configuration, advanced step by step."""
+
+    def __init__(self, cfg: syn.NosaConfig, pool_k: np.ndarray, pool_v: np.ndarray,
+                 resident: Optional[np.ndarray] = None, lib_path: Optional[str] = None):
+        self.cfg = cfg
+        self.L = load(lib_path)
+        c = cfg
+        NG, nb = c.B * c.Hkv, c.max_blocks
+        self.c = OrcCfg(c.B, c.Hq, c.Hkv, c.d, c.block, c.sub_block, c.k_q, c.k_e, c.rows, nb,
+                        c.n_slots, int(c.offload), c.scale)
+        self.K = np.ascontiguousarray(pool_k).copy()
+        self.V = np.ascontiguousarray(pool_v).copy()
+        self.kbar = np.zeros((NG, c.max_sub, c.d), np.float64)
+        self.len = np.zeros(NG, np.int32)
+        self.prev_sel = np.zeros((NG, nb), np.uint8)
+        self.alive = np.zeros((NG, nb), np.uint8)
+        self.block_slot = np.full((NG, nb), -1, np.int32)
+        self.slot_owner = np.full((NG, c.n_slots), -1, np.int32)
+        self.last_used = np.zeros((NG, nb), np.int32)
+        self.st = OrcState(*[_p(a) for a in (self.K, self.V, self.kbar, self.len, self.prev_sel,
+                                              self.alive, self.block_slot, self.slot_owner,
+                                              self.last_used)])
+        T = np.ascontiguousarray(np.array(c.T, np.int32))
+        res = None if resident is None else np.ascontiguousarray(resident, np.uint8)
+        rc = self.L.orc_init(ctypes.byref(self.c), ctypes.byref(self.st), _p(T), _p(res))
+        if rc != 0:
+            raise ValueError(f"orc_init failed ({rc})")
+
+    def append(self, k_new, v_new):
+        self.L.orc_append(ctypes.byref(self.c), ctypes.byref(self.st),
+                          _p(np.ascontiguousarray(k_new)), _p(np.ascontiguousarray(v_new)))
+
+    def block_scores(self, rows: np.ndarray) -> np.ndarray:
+        c = self.cfg
+        out = np.empty((c.B * c.Hkv, c.max_blocks), np.float64)
+        self.L.orc_block_scores(ctypes.byref(self.c), ctypes.byref(self.st),
+                                _p(np.ascontiguousarray(rows)), _p(out))
+        return out
+
+    def select(self, scores, evict, commit=True):
+        c = self.cfg
+        NG = c.B * c.Hkv
+        sel = np.empty((NG, c.k), np.int32)
+        src = np.empty((NG, c.k), np.int8)
+        gap = np.empty(NG, np.float64)
+        self.L.orc_select(ctypes.byref(self.c), ctypes.byref(self.st),
+                          _p(np.ascontiguousarray(scores, np.float64)),
+                          _p(np.ascontiguousarray(evict, np.float32)), _p(sel), _p(src), _p(gap),
+                          int(commit))
+        return sel, src, gap
+
+    def residency(self, sel):
+        mc = np.zeros(self.cfg.B * self.cfg.Hkv, np.int32)
+        rc = self.L.orc_residency(ctypes.byref(self.c), ctypes.byref(self.st),
+                                  _p(np.ascontiguousarray(sel, np.int32)), _p(mc))
+        if rc != 0:
+            raise RuntimeError("oracle residency: no victim available")
+        return mc
+
+    def attend(self, q, sel):
+        c = self.cfg
+        out = np.empty((c.B, c.Hq, c.d), np.float64)
+        self.L.orc_attend(ctypes.byref(self.c), ctypes.byref(self.st),
+                          _p(np.ascontiguousarray(q)), _p(np.ascontiguousarray(sel, np.int32)),
+                          _p(out))
+        return out
+
+    def snapshot(self) -> dict:
+        return {k: getattr(self, k).copy() for k in
+                ("len", "prev_sel", "alive", "block_slot", "slot_owner", "last_used")}
+
+
+@dataclass
+class StepRecord:
+    q: np.ndarray               # uint16 [B][Hq][d]
+    rows: np.ndarray            # uint16 [B][Hkv][R][d] scoring rows (q regrouped or forecast)
+    forecast: Optional[np.ndarray]
+    scores: np.ndarray          # fp64 [B*Hkv][max_blocks]
+    sel: np.ndarray             # int32 [B*Hkv][k]
+    src: np.ndarray             # int8
+    gap: np.ndarray             # fp64 [B*Hkv]
+    miss: np.ndarray            # int32 [B*Hkv]
+    out: np.ndarray             # fp64 [B][Hq][d]
+    retries: np.ndarray         # int [B][Hkv]
+    state: dict = field(default_factory=dict)
+
+
+@dataclass
+class Case:
+    cfg: syn.NosaConfig
+    inputs: syn.Inputs
+    steps: List[StepRecord]
+
+
+def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = MARGIN,
+             max_retry: int = 64, keep_state: bool = True, lib_path: Optional[str] = None) -> Case:
+    """Generate a config's inputs and run the oracle over its steps.
+
+    Margin enforcement: after each append the query-aware cut of every group is
+    checked; when the fp64 gap between the last selected and the first
+    unselected block score is below `margin`, that group's query (or forecast)
+    row is redrawn from the next retry stream. The final inputs are the ones
+    recorded, so the GPU and the oracle consume identical arrays.
+    """
+    inp = syn.make_inputs(cfg)
+    orc = Oracle(cfg, inp.pool_k, inp.pool_v, inp.resident, lib_path)
+    S = cfg.steps if steps is None else steps
+    G, R = cfg.G, cfg.rows
+    prev = None
+    recs = []
+    for t in range(S):
+        orc.append(inp.k_new[t], inp.v_new[t])
+        retry = np.zeros((cfg.B, cfg.Hkv), np.int64)
+        pending = np.ones((cfg.B, cfg.Hkv), bool)
+        while True:
+            qs = syn.query_step(cfg, t, prev, retry)
+            q16 = syn.round_bf16(qs)
+            fc = None
+            if cfg.n_score_rows == 1:
+                fc = syn.round_bf16(syn.forecast_step(cfg, t, retry))
+                rows = fc.reshape(cfg.B, cfg.Hkv, 1, cfg.d)
+            else:
+                rows = q16.reshape(cfg.B, cfg.Hkv, G, cfg.d)
+            scores = orc.block_scores(rows)
+            _, _, gap = orc.select(scores, inp.evict[t], commit=False)
+            bad = (gap.reshape(cfg.B, cfg.Hkv) < margin) & pending
+            if not bad.any():
+                break
+            if (retry[bad] >= max_retry).any():
+                raise RuntimeError(f"{cfg.name}: no query with margin {margin} at step {t}")
+            retry[bad] += 1
+        prev = qs
+        sel, src, gap = orc.select(scores, inp.evict[t], commit=True)
+        miss = orc.residency(sel)
+        out = orc.attend(q16, sel)
+        recs.append(StepRecord(q16, np.ascontiguousarray(rows), fc, scores, sel, src, gap, miss, out,
+                               retry, orc.snapshot() if keep_state else {}))
+    case = Case(cfg, inp, recs)
+    case.oracle = orc
+    return case

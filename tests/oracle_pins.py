@@ -1,0 +1,295 @@
+"""Checks that pin the fp64 oracle to things other than itself.
+
+Each ``check_*`` takes an oracle library path (so the mutation test can run the
+same checks against deliberately broken copies of the oracle) and raises
+AssertionError on a mismatch. What pins what:
+
+* pooling          - torch's avg_pool1d / max_pool1d applied to token-level logits
+                     (linearity: mean of q.K over a sub-block = q . mean K)
+* top-m            - O(n^2) rank counting on small inputs with many ties
+* dual selection   - a hand-worked example (golden fixture) and the pages'
+                     invariants on generated traces (never-again, locality bound,
+                     disjointness, |S| = min(k, N)), brute-force top-m of each set
+* closed form      - static eviction scores with no new block: Gamma_e is the
+                     fixed top-k_e of the prefill blocks at every step
+* attention        - torch's scaled_dot_product_attention (fp64) when every block
+                     is selected; torch.softmax over gathered tokens otherwise
+* residency        - a hand-worked example (golden fixture) and invariants
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+import nosa_synth as syn
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _tokens(case_or_orc, gi, L):
+    orc = case_or_orc
+    K = syn.bf16_to_f64(orc.K[gi // orc.cfg.Hkv, gi % orc.cfg.Hkv, :L])
+    V = syn.bf16_to_f64(orc.V[gi // orc.cfg.Hkv, gi % orc.cfg.Hkv, :L])
+    return K, V
+
+
+# ----------------------------------------------------------------- top-m
+def check_topm_bruteforce(lib_path=None, trials=300, seed=0):
+    L = O.load(lib_path)
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        n = int(rng.integers(1, 40))
+        key = rng.integers(0, 6, n).astype(np.float64)  # many ties
+        cand = (rng.random(n) < 0.7).astype(np.uint8)
+        m = int(rng.integers(0, n + 2))
+        ch, gap = O.topm(key, cand, m, L)
+        idx = np.flatnonzero(cand)
+        want = np.zeros(n, np.uint8)
+        for j in idx:
+            rank = sum(1 for i in idx if key[i] > key[j] or (key[i] == key[j] and i < j))
+            if rank < m:
+                want[j] = 1
+        assert np.array_equal(ch, want), (key, cand, m, ch, want)
+        take = min(m, idx.size)
+        if 1 <= take < idx.size:
+            ordered = sorted(idx, key=lambda j: sum(1 for i in idx if key[i] > key[j] or (key[i] == key[j] and i < j)))
+            assert gap == key[ordered[take - 1]] - key[ordered[take]]
+        else:
+            assert gap == np.inf
+
+
+# ----------------------------------------------------------------- pooling
+def check_pooling_library(cfg, lib_path=None, steps=3):
+    """Block scores = max_pool(avg_pool(mean_r sigma q_r . K_tau)) via torch routines."""
+    case = O.run_case(cfg, steps=steps, lib_path=lib_path)
+    orc = case.oracle
+    c = cfg
+    # re-run: scores were recorded per step; recompute from the final oracle token store
+    for t, rec in enumerate(case.steps):
+        for gi in range(c.B * c.Hkv):
+            b = gi // c.Hkv
+            Lt = c.T[b] + t + 1
+            K, _ = _tokens(orc, gi, Lt)
+            rows = syn.bf16_to_f64(rec.rows.reshape(c.B * c.Hkv, c.rows, c.d)[gi])
+            logit = c.scale * (torch.from_numpy(rows) @ torch.from_numpy(K).T)  # [R][L]
+            u_tok = logit.mean(0).view(1, 1, -1)
+            u_sub = F.avg_pool1d(u_tok, c.sub_block, c.sub_block, ceil_mode=True)
+            spb = c.block // c.sub_block
+            s_blk = F.max_pool1d(u_sub, spb, spb, ceil_mode=True).view(-1).numpy()
+            N = -(-Lt // c.block)
+            got = rec.scores[gi]
+            assert s_blk.size == N
+            np.testing.assert_allclose(got[:N], s_blk, rtol=1e-12, atol=1e-12)
+            assert np.all(np.isneginf(got[N:]))
+
+
+# ----------------------------------------------------------------- selection
+def _sets(rec, gi):
+    sel, src = rec.sel[gi], rec.src[gi]
+    S = [int(j) for j in sel if j >= 0]
+    Ge = {int(j) for j, s in zip(sel, src) if s == 1}
+    Gq = {int(j) for j, s in zip(sel, src) if s == 2}
+    return S, Ge, Gq
+
+
+def _brute_top(keys: dict, m: int):
+    items = list(keys.items())
+    out = set()
+    for j, v in items:
+        rank = sum(1 for i, w in items if w > v or (w == v and i < j))
+        if rank < m:
+            out.add(j)
+    return out
+
+
+def check_selection_trace(case):
+    """The pages' invariants plus brute-force top-m of each set on a generated trace."""
+    c = case.cfg
+    for gi in range(c.B * c.Hkv):
+        b = gi // c.Hkv
+        n0 = -(-c.T[b] // c.block)
+        prev = set(range(n0))
+        dropped = set()      # blocks that were in S(t-1) but not kept by Gamma_e(t)
+        for t, rec in enumerate(case.steps):
+            Lt = c.T[b] + t + 1
+            N = -(-Lt // c.block)
+            S, Ge, Gq = _sets(rec, gi)
+            assert S == sorted(set(S)), "S ascending and unique"
+            assert len(S) == min(c.k, N), (len(S), c.k, N)
+            assert not (Ge & Gq), "Gamma_e and Gamma_q disjoint"
+            assert Ge | Gq == set(S)
+            assert Ge <= prev, "Gamma_e drawn from S(t-1)"
+            assert not (Ge & dropped), "a block left out by Gamma_e never returns to it"
+            if len(Ge) == c.k_e:
+                assert len(set(S) & prev) >= c.k_e, "locality gamma(t) >= k_e/k"
+            if n0 >= c.k_e:
+                assert len(Ge) == c.k_e
+            # Gamma_e = brute-force top of the eviction scores over its candidates
+            cand_e = prev - dropped
+            ev = rec_evict(case, t)[gi]
+            assert Ge == _brute_top({j: float(ev[j]) for j in cand_e}, c.k_e)
+            # Gamma_q = brute-force top of block scores over the rest
+            rest = {j: float(rec.scores[gi][j]) for j in range(N) if j not in Ge}
+            assert Gq == _brute_top(rest, min(c.k - len(Ge), N - len(Ge)))
+            dropped |= (cand_e - Ge)
+            prev = set(S)
+
+
+def rec_evict(case, t):
+    c = case.cfg
+    return case.inputs.evict[t].reshape(c.B * c.Hkv, c.max_blocks)
+
+
+def check_static_closed_form(lib_path=None):
+    """Static eviction scores, no block created: Gamma_e(t) = top-k_e over prefill blocks."""
+    cfg = syn.configs()["tiny_static"]
+    assert cfg.drift == 0 and (cfg.T[0] + cfg.steps - 1) // cfg.block == (cfg.T[0] - 1) // cfg.block
+    case = O.run_case(cfg, lib_path=lib_path)
+    n0 = -(-cfg.T[0] // cfg.block)
+    for gi in range(cfg.B * cfg.Hkv):
+        e = rec_evict(case, 0)[gi][:n0].astype(np.float64)
+        order = np.lexsort((np.arange(n0), -e))     # score descending, index ascending
+        want = set(int(j) for j in order[:cfg.k_e])
+        for rec in case.steps:
+            _, Ge, _ = _sets(rec, gi)
+            assert Ge == want
+
+
+def _hand_cfg(h):
+    c = h["config"]
+    return syn.NosaConfig("hand", c["B"], c["Hq"], c["Hkv"], c["d"], (c["T"],), c["block"],
+                          c["sub_block"], c["k_q"], c["k_e"], c["steps"], slots=c.get("slots", 0),
+                          cfg_id=999)
+
+
+def check_hand_dual_selection(lib_path=None):
+    h = json.load(open(os.path.join(GOLDEN, "hand_dual_selection.json")))
+    cfg = _hand_cfg(h)
+    nb = cfg.max_blocks
+    z = np.zeros((1, 1, nb * cfg.block, cfg.d), np.uint16)
+    orc = O.Oracle(cfg, z, z, None, lib_path)
+    kn = np.zeros((1, 1, cfg.d), np.uint16)
+    for t in range(cfg.steps):
+        orc.append(kn, kn)
+        N = -(-(cfg.T[0] + t + 1) // cfg.block)
+        sc = np.full((1, nb), -np.inf)
+        sc[0, :len(h["scores"][t])] = h["scores"][t]
+        ev = np.zeros((1, nb), np.float32)
+        ev[0, :len(h["evict"][t])] = h["evict"][t]
+        sel, src, _ = orc.select(sc, ev)
+        got = [int(j) for j in sel[0] if j >= 0]
+        assert got == h["expect_sel"][t], (t, got)
+        assert sorted(int(j) for j, s in zip(sel[0], src[0]) if s == 1) == h["expect_gamma_e"][t]
+        assert [j for j in range(N) if orc.alive[0, j]] == h["expect_alive_below_N"][t]
+
+
+def check_hand_residency(lib_path=None):
+    h = json.load(open(os.path.join(GOLDEN, "hand_residency.json")))
+    cfg = _hand_cfg(h)
+    nb = cfg.max_blocks
+    z = np.zeros((1, 1, nb * cfg.block, cfg.d), np.uint16)
+    res = np.zeros((1, 1, nb), np.uint8)
+    res[0, 0, h["resident"]] = 1
+    orc = O.Oracle(cfg, z, z, res, lib_path)
+    kn = np.zeros((1, 1, cfg.d), np.uint16)
+    for t in range(cfg.steps):
+        orc.append(kn, kn)
+        sc = np.array([h["scores"][t]], np.float64)
+        ev = np.array([h["evict"][t]], np.float32)
+        sel, _, _ = orc.select(sc, ev)
+        assert [int(j) for j in sel[0] if j >= 0] == h["expect_sel"][t]
+        mc = orc.residency(sel)
+        assert int(mc[0]) == h["expect_miss"][t], (t, mc)
+        assert orc.block_slot[0].tolist() == h["expect_block_slot"][t], (t, orc.block_slot[0])
+        assert orc.slot_owner[0].tolist() == h["expect_slot_owner"][t]
+        assert orc.last_used[0].tolist() == h["expect_last_used"][t]
+
+
+def check_residency_trace(case):
+    """Invariants of the residency model on a generated offload trace."""
+    c = case.cfg
+    for t, rec in enumerate(case.steps):
+        st = rec.state
+        for gi in range(c.B * c.Hkv):
+            b = gi // c.Hkv
+            Lt = c.T[b] + t + 1
+            tail = (Lt - 1) // c.block
+            S = [int(j) for j in rec.sel[gi] if j >= 0]
+            bsl, own = st["block_slot"][gi], st["slot_owner"][gi]
+            for j in S + [tail]:
+                assert bsl[j] >= 0, "selected blocks and the tail are resident"
+                assert st["last_used"][gi][j] == Lt
+            res = [j for j in range(c.max_blocks) if bsl[j] >= 0]
+            assert len(res) <= c.slots
+            for j in res:
+                assert own[bsl[j]] == j, "slot table is the inverse of the block table"
+            assert sum(1 for z in own if z >= 0) == len(res)
+            if t >= 1:
+                # Gamma_e is inside S(t-1), which was resident: only Gamma_q (and a new tail) miss
+                assert rec.miss[gi] <= c.k_q + 1
+
+
+# ----------------------------------------------------------------- attention
+def _attn_ref(orc, rec, gi, Lt, all_tokens=False):
+    c = orc.cfg
+    K, V = _tokens(orc, gi, Lt)
+    if all_tokens:
+        idx = np.arange(Lt)
+    else:
+        blocks = [int(j) for j in rec.sel[gi] if j >= 0]
+        idx = np.concatenate([np.arange(j * c.block, min((j + 1) * c.block, Lt)) for j in blocks])
+    b, g = gi // c.Hkv, gi % c.Hkv
+    q = syn.bf16_to_f64(rec.q[b, g * c.G:(g + 1) * c.G])
+    return torch.from_numpy(q), torch.from_numpy(K[idx]), torch.from_numpy(V[idx])
+
+
+def check_attention_dense_sdpa(lib_path=None):
+    """With every block selected the step is plain softmax attention (torch SDPA)."""
+    cfg = syn.configs()["tiny_dense"]
+    case = O.run_case(cfg, lib_path=lib_path)
+    orc = case.oracle
+    for t, rec in enumerate(case.steps):
+        for gi in range(cfg.B * cfg.Hkv):
+            Lt = cfg.T[0] + t + 1
+            N = -(-Lt // cfg.block)
+            assert [int(j) for j in rec.sel[gi] if j >= 0] == list(range(N))
+            q, K, V = _attn_ref(orc, rec, gi, Lt, all_tokens=True)
+            ref = F.scaled_dot_product_attention(q[None, :, None, :], K[None, None].expand(1, cfg.G, -1, -1),
+                                                 V[None, None].expand(1, cfg.G, -1, -1),
+                                                 scale=cfg.scale)[0, :, 0, :].numpy()
+            b, g = gi // cfg.Hkv, gi % cfg.Hkv
+            np.testing.assert_allclose(rec.out[b, g * cfg.G:(g + 1) * cfg.G], ref, rtol=1e-11, atol=1e-13)
+
+
+def check_attention_subset(cfg, lib_path=None, steps=None):
+    case = O.run_case(cfg, steps=steps, lib_path=lib_path)
+    orc = case.oracle
+    for t, rec in enumerate(case.steps):
+        for gi in range(cfg.B * cfg.Hkv):
+            Lt = cfg.T[gi // cfg.Hkv] + t + 1
+            q, K, V = _attn_ref(orc, rec, gi, Lt)
+            ref = (torch.softmax(cfg.scale * q @ K.T, dim=-1) @ V).numpy()
+            b, g = gi // cfg.Hkv, gi % cfg.Hkv
+            np.testing.assert_allclose(rec.out[b, g * cfg.G:(g + 1) * cfg.G], ref, rtol=1e-11, atol=1e-13)
+    return case
+
+
+def run_all(lib_path=None):
+    cs = syn.configs()
+    check_topm_bruteforce(lib_path, trials=120)
+    check_hand_dual_selection(lib_path)
+    check_hand_residency(lib_path)
+    check_static_closed_form(lib_path)
+    check_attention_dense_sdpa(lib_path)
+    for name in ("ragged", "tiny_forecast", "bs128_d64"):
+        check_pooling_library(cs[name], lib_path, steps=2)
+    for name in ("ragged", "ragged_offload", "g8"):
+        case = check_attention_subset(cs[name], lib_path)
+        check_selection_trace(case)
+        if case.cfg.offload:
+            check_residency_trace(case)
