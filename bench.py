@@ -1,0 +1,392 @@
+"""Benchmark of one NOSA sparse-decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama] [--impl reference]
+
+One step = append -> pooled block scores -> dual selection -> (gather) -> split-K
+attention + combine for every GQA group of the workload, through the C ABI
+(nosa_step). Default workload: a Llama-3.1-8B-shaped attention layer (B=16,
+Hq=32, Hkv=8, d=128, T=32768, block 64, sub-block 16, k=64 with k_q=16 and
+k_e=48, 8 planted high-affinity blocks per group), synthetic seeded inputs.
+
+Printed: one JSON line. `value` is queries/s (query-head vectors, B*Hq per
+step, summed over ranks) from CUDA-event time of the timed steps, inputs
+resident in HBM, L2 flushed (256 MiB write) before every timed step. `e2e` is
+the same metric with each step's inputs copied from pinned host memory and the
+outputs copied back inside the timed region. `roofline` is for the attention
+kernel (the largest share of the step), `cpu_baseline` times the fp64 oracle on
+a bounded sample of the same workload on this host's cores.
+
+--impl reference times the oracle itself (the only reference implementation
+that exists for this method) and prints the same JSON line with impl=reference.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import nosa_synth as syn  # noqa: E402
+
+METRIC = "sparse decode attn: queries/s, step µs, achieved HBM GB/s (% of peak)"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def workload(name: str, steps: int) -> syn.NosaConfig:
+    base = syn.configs()[name]
+    return base.with_(steps=steps)
+
+
+def describe(cfg: syn.NosaConfig) -> str:
+    return (f"{cfg.name}: B={cfg.B} Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} T={cfg.T[0]} "
+            f"block={cfg.block} sub_block={cfg.sub_block} k={cfg.k} (k_q={cfg.k_q}, k_e={cfg.k_e})"
+            + (f" slots={cfg.slots} offload" if cfg.offload else " all KV in HBM"))
+
+
+def step_bytes(cfg: syn.NosaConfig, L: int):
+    """Algorithmic bytes of one step at context length L (after the append), per step.
+
+    Returns (total, attention kernel, score/select kernel)."""
+    NG, G, d, bs = cfg.B * cfg.Hkv, cfg.G, cfg.d, cfg.block
+    N = -(-L // bs)
+    M = -(-L // cfg.sub_block)
+    nsel = min(cfg.k, N)
+    tail_tokens = L - (N - 1) * bs
+    # K and V of the selected blocks; the tail block (always among them once k >= N) at its
+    # present tokens only when it is selected -- counted as full pages otherwise
+    kv = nsel * bs * d * 2 * 2
+    attn = NG * (kv + G * d * 2 + G * d * 4 + cfg.k * 4 + cfg.k * 4)
+    score = NG * (M * d * 4 + N * 4 + 2 * 2 * 4 * (-(-N // 32)) + cfg.rows * d * 2
+                  + 2 * d * 2 + N * 4 * 2 + cfg.k * 4)
+    return attn + score, attn, score
+
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.p = None
+        self.path = os.path.join("/tmp", f"nosa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.p is not None:
+            time.sleep(0.2)
+            self.p.terminate()
+            self.p.wait()
+            self.f.close()
+
+    def summary(self):
+        if self.p is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(cfg: syn.NosaConfig, steps: int, budget_s: float = 20.0):
+    """Times the fp64 oracle (append, score, select, residency, attention) on a bounded
+    sample of the workload: the first batch entries of the same layer, `steps` decode steps."""
+    import oracle as O
+    B_s = max(1, min(cfg.B, 2))
+    sub = cfg.with_(name=cfg.name + "_sample", B=B_s, T=cfg.T[:B_s], steps=steps)
+    inp = syn.make_inputs(sub)
+    orc = O.Oracle(sub, inp.pool_k, inp.pool_v, inp.resident)
+    prev = None
+    zero = np.zeros((sub.B, sub.Hkv), np.int64)
+    qs_all = []
+    for t in range(steps):
+        prev = syn.query_step(sub, t, prev, zero)
+        qs_all.append(syn.round_bf16(prev))
+    times = []
+    for t in range(steps):
+        q16 = qs_all[t]
+        t0 = time.perf_counter()
+        orc.append(inp.k_new[t], inp.v_new[t])
+        rows = q16.reshape(sub.B, sub.Hkv, sub.G, sub.d)
+        sc = orc.block_scores(rows)
+        sel, _, _ = orc.select(sc, inp.evict[t])
+        orc.residency(sel)
+        orc.attend(q16, sel)
+        times.append(time.perf_counter() - t0)
+        if sum(times) > budget_s:
+            break
+    n = len(times)
+    tot = sum(times)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": sub.B * sub.Hq * n / tot, "unit": "queries/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} decode steps of {B_s} of {cfg.B} batch entries of the same layer "
+                      f"(fp64 C oracle, OpenMP over groups), {tot:.2f} s"}, times
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps = args.warmup + args.steps
+    res, times = oracle_sample(cfg, steps, budget_s=1e9)
+    timed = times[args.warmup:]
+    B_s = max(1, min(cfg.B, 2))
+    val = B_s * cfg.Hq * len(timed) / sum(timed)
+    cb = dict(res)
+    cb["value"] = val
+    cb["sample"] = f"{len(timed)} timed decode steps (+{args.warmup} warm-up) of {B_s} of {cfg.B} batch entries"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "queries/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(timed) / len(timed), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(cfg), "sample_batch": B_s},
+            "cpu_baseline": cb,
+            "e2e": {"value": val, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args, cfg):
+    import torch
+    import torch.distributed as dist
+    import kv_cache_offload_nosa_b200 as nosa
+    from kv_cache_offload_nosa_b200 import build as nb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    nb.build()
+    # each rank is an independent replica with its own seeded batch (weak scaling)
+    if world > 1:
+        cfg = cfg.with_(cfg_id=cfg.cfg_id + 1000 * rank)
+    n_e2e = args.e2e_steps
+    n_prof = 3
+    total_steps = args.warmup + args.steps + n_prof + n_e2e
+    cfg = cfg.with_(steps=total_steps)
+    inp = syn.make_inputs(cfg)
+    NG = cfg.B * cfg.Hkv
+    cc = nosa.make_config(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.block, cfg.sub_block, cfg.k_q, cfg.k_e,
+                          cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows, scale=cfg.scale)
+    cache = nosa.NosaCache(cc, offload=cfg.offload)
+    pk = torch.from_numpy(inp.pool_k.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)
+    pv = torch.from_numpy(inp.pool_v.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)
+    resident = None
+    if cfg.offload:
+        cache.pool_view("host_k").copy_(pk)
+        cache.pool_view("host_v").copy_(pv)
+        resident = torch.from_numpy(inp.resident.reshape(NG, -1)).cuda()
+    else:
+        cache.pool_view("k_pool").copy_(pk)
+        cache.pool_view("v_pool").copy_(pv)
+    del pk, pv
+    inp.pool_k = inp.pool_v = None
+    plen = torch.tensor(cfg.T, dtype=torch.int32, device="cuda")
+    cache.init(plen, resident)
+    # per-step inputs (queries follow the workload's process, no margin redraws)
+    prev, zero = None, np.zeros((cfg.B, cfg.Hkv), np.int64)
+    qs = []
+    for t in range(total_steps):
+        prev = syn.query_step(cfg, t, prev, zero)
+        qs.append(syn.round_bf16(prev))
+    h_q = torch.from_numpy(np.stack(qs)).view(torch.int16)
+    h_kn = torch.from_numpy(inp.k_new).view(torch.int16)
+    h_vn = torch.from_numpy(inp.v_new).view(torch.int16)
+    h_ev = torch.from_numpy(inp.evict)
+    d_q, d_kn, d_vn, d_ev = (x.cuda() for x in (h_q, h_kn, h_vn, h_ev))
+    sel = torch.empty(NG * cfg.k, dtype=torch.int32, device="cuda")
+    out = torch.empty(cfg.B * cfg.Hq * cfg.d, dtype=torch.float32, device="cuda")
+    miss = torch.empty(NG, dtype=torch.int32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def do_step(t, events=None):
+        cache.step(d_q[t], d_kn[t], d_vn[t], d_ev[t], sel, out, miss, stream=stream, events=events)
+
+    t = 0
+    for _ in range(args.warmup):
+        do_step(t)
+        t += 1
+    torch.cuda.synchronize()
+    rc, err = cache.check()
+    if rc != 0:
+        raise RuntimeError(f"device fault after warm-up: rc={rc} err={err}")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    Ls = []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            do_step(t)
+            ends[i].record(stream)
+            Ls.append(cfg.T[0] + t + 1)
+            t += 1
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    tot_ms = sum(step_ms)
+    # per-kernel times of the same step (instrumented steps, events between kernels)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_prof)]
+    for e4 in evs:
+        for e in e4:
+            e.record(stream)
+    torch.cuda.synchronize()
+    prof_L = []
+    for i in range(n_prof):
+        flush.zero_()
+        do_step(t, events=evs[i])
+        prof_L.append(cfg.T[0] + t + 1)
+        t += 1
+    torch.cuda.synchronize()
+    k_score = [e[0].elapsed_time(e[1]) for e in evs]
+    k_gather = [e[1].elapsed_time(e[2]) for e in evs]
+    k_attn = [e[2].elapsed_time(e[3]) for e in evs]
+    # end to end: pinned host inputs in, outputs back, inside the timed region
+    hp = [x.pin_memory() for x in (h_q, h_kn, h_vn, h_ev)]
+    o_host = torch.empty(out.numel(), dtype=torch.float32, pin_memory=True)
+    s_host = torch.empty(sel.numel(), dtype=torch.int32, pin_memory=True)
+    m_host = torch.empty(miss.numel(), dtype=torch.int32, pin_memory=True)
+    bq, bk, bv, be = (torch.empty_like(x[0], device="cuda") for x in hp)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(n_e2e):
+        bq.copy_(hp[0][t], non_blocking=True)
+        bk.copy_(hp[1][t], non_blocking=True)
+        bv.copy_(hp[2][t], non_blocking=True)
+        be.copy_(hp[3][t], non_blocking=True)
+        cache.step(bq, bk, bv, be, sel, out, miss, stream=stream)
+        o_host.copy_(out, non_blocking=True)
+        s_host.copy_(sel, non_blocking=True)
+        m_host.copy_(miss, non_blocking=True)
+        t += 1
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    rc, err = cache.check()
+    if rc != 0:
+        raise RuntimeError(f"device fault in timed steps: rc={rc} err={err}")
+
+    # max over ranks
+    agg = torch.tensor([tot_ms, e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(agg, op=dist.ReduceOp.MAX)
+    tot_ms, e2e_ms = agg.tolist()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    q_per_step = cfg.B * cfg.Hq * world
+    value = q_per_step * args.steps / (tot_ms / 1e3)
+    hbm_peak, peak_kind = peaks()
+    step_b = [step_bytes(cfg, L)[0] for L in Ls]
+    hbm_gbs = sum(step_b) / (tot_ms / 1e3) / 1e9
+    attn_b = [step_bytes(cfg, L)[1] for L in prof_L]
+    attn_ms = float(np.mean(k_attn))
+    achieved = float(np.mean(attn_b)) / (attn_ms / 1e3) / 1e9
+    clocks = clk.summary()
+    h2d = sum(x[0].numel() * x.element_size() for x in hp)
+    d2h = o_host.numel() * 4 + s_host.numel() * 4 + m_host.numel() * 4
+    line = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(cfg), "global_batch": cfg.B * world, "seq_len": cfg.T[0],
+                   "parallelism": f"replicas x{world} (batch-sharded, no collective)",
+                   "l2": "flushed (256 MiB write) before every timed step",
+                   "queries_per_step": q_per_step},
+        "step_us": 1e3 * tot_ms / args.steps,
+        "step_us_median": 1e3 * float(np.median(step_ms)),
+        "hbm_gbs": hbm_gbs, "hbm_frac": hbm_gbs / hbm_peak,
+        "bytes_per_step": float(np.mean(step_b)),
+        "kernel_us": {"score_select": 1e3 * float(np.mean(k_score)),
+                      "gather": 1e3 * float(np.mean(k_gather)), "attention": 1e3 * attn_ms},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "attn_kernel",
+                     "peak_kind": peak_kind,
+                     "bytes_per_launch": float(np.mean(attn_b))},
+        "e2e": {"value": q_per_step / (e2e_ms / 1e3), "unit": "queries/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * (3 if cfg.offload else 2),
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        cb, _ = oracle_sample(workload(args.workload, 4), 3, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = cb
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = workload(args.workload, args.warmup + args.steps)
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_gpu(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+"""Python binding of libnosa.so: one NOSA sparse-decode step on a B200.
+
+Argument marshalling only. Every step of the path (append, pooled scoring,
+dual selection, residency and UVA gather, split-K attention and combine) runs
+in the CUDA kernels of ``libnosa.so``; there is no CPU or PyTorch fallback, and
+loading fails loudly when the library is missing. PyTorch provides device
+memory, pinned host memory and streams.
+
+The function names mirror the C ABI of ``include/nosa.h``; tensors are passed
+by their data pointers and must already have the documented dtype, shape and
+placement.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnosa.so")
+
+NOSA_OK, NOSA_EINVAL, NOSA_ENOMEM, NOSA_ECUDA, NOSA_EDEVICE, NOSA_ETIMEOUT = range(6)
+ERR_BLOCK_TABLE, ERR_SEL, ERR_NO_VICTIM, ERR_TIMEOUT, ERR_FULL, ERR_INIT = 1, 2, 4, 8, 16, 32
+
+EXPORTS = ("nosa_state_sizes", "nosa_workspace_size", "nosa_workspace_init", "nosa_state_init",
+           "nosa_append", "nosa_score_blocks", "nosa_select", "nosa_gather", "nosa_decode_attn",
+           "nosa_step", "nosa_check_device", "nosa_status_string", "nosa_last_error")
+
+
+class nosa_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "Hq", "Hkv", "d", "block_size", "sub_block", "k_q", "k_e", "max_blocks",
+                 "slots", "n_score_rows", "attn_split")] + [("scale", ctypes.c_float)]
+
+
+STATE_FIELDS = ("seq_len", "kc", "prev_sel", "alive", "last_used", "block_table", "slot_owner",
+                "k_pool", "v_pool", "host_k", "host_v", "err")
+
+
+class nosa_state(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in STATE_FIELDS]
+
+
+class nosa_sizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in STATE_FIELDS]
+
+
+class NosaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"nosa status {status}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: Optional[str] = None):
+    """Loads libnosa.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"libnosa.so not built at {p}; run kv_cache_offload_nosa_b200/build.py")
+    L = ctypes.CDLL(p)
+    vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    cfgp, stp = ctypes.POINTER(nosa_config), ctypes.POINTER(nosa_state)
+    sig = {
+        "nosa_state_sizes": [cfgp, ctypes.POINTER(nosa_sizes)],
+        "nosa_workspace_size": [cfgp, ctypes.POINTER(ctypes.c_size_t)],
+        "nosa_workspace_init": [vp, sz, vp],
+        "nosa_state_init": [cfgp, stp, vp, vp, vp, sz, vp],
+        "nosa_append": [cfgp, stp, vp, vp, vp],
+        "nosa_score_blocks": [cfgp, stp, vp, vp, vp],
+        "nosa_select": [cfgp, stp, vp, vp, vp, vp],
+        "nosa_gather": [cfgp, stp, vp, vp, vp, sz, vp],
+        "nosa_decode_attn": [cfgp, stp, vp, vp, vp, vp, sz, vp],
+        "nosa_step": [cfgp, stp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp],
+        "nosa_check_device": [stp, vp, ctypes.POINTER(ctypes.c_uint32)],
+    }
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = i32
+    L.nosa_status_string.argtypes = [i32]
+    L.nosa_status_string.restype = ctypes.c_char_p
+    L.nosa_last_error.argtypes = []
+    L.nosa_last_error.restype = ctypes.c_char_p
+    if path is None:
+        _lib = L
+    return L
+
+
+def _check(rc: int):
+    if rc != NOSA_OK:
+        L = load()
+        raise NosaError(rc, f"{L.nosa_status_string(rc).decode()}: {L.nosa_last_error().decode()}")
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_config(B, Hq, Hkv, d, block_size, sub_block, k_q, k_e, max_blocks, slots=None,
+                n_score_rows=None, attn_split=0, scale=None) -> nosa_config:
+    G = Hq // Hkv
+    return nosa_config(B, Hq, Hkv, d, block_size, sub_block, k_q, k_e, max_blocks,
+                       max_blocks if slots is None else slots, G if n_score_rows is None else n_score_rows,
+                       attn_split, (1.0 / d ** 0.5) if scale is None else scale)
+
+
+def state_sizes(cfg: nosa_config) -> nosa_sizes:
+    s = nosa_sizes()
+    _check(load().nosa_state_sizes(ctypes.byref(cfg), ctypes.byref(s)))
+    return s
+
+
+def workspace_size(cfg: nosa_config) -> int:
+    n = ctypes.c_size_t()
+    _check(load().nosa_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def workspace_init(ws, nbytes: int, stream=None):
+    _check(load().nosa_workspace_init(_ptr(ws), nbytes, _stream(stream)))
+
+
+def state_init(cfg, st: nosa_state, prefill_len, resident, ws, ws_bytes, stream=None):
+    _check(load().nosa_state_init(ctypes.byref(cfg), ctypes.byref(st), _ptr(prefill_len),
+                                  _ptr(resident), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def append(cfg, st, k_new, v_new, stream=None):
+    _check(load().nosa_append(ctypes.byref(cfg), ctypes.byref(st), _ptr(k_new), _ptr(v_new),
+                              _stream(stream)))
+
+
+def score_blocks(cfg, st, rows, block_scores, stream=None):
+    _check(load().nosa_score_blocks(ctypes.byref(cfg), ctypes.byref(st), _ptr(rows),
+                                    _ptr(block_scores), _stream(stream)))
+
+
+def select(cfg, st, block_scores, evict, sel, stream=None):
+    _check(load().nosa_select(ctypes.byref(cfg), ctypes.byref(st), _ptr(block_scores), _ptr(evict),
+                              _ptr(sel), _stream(stream)))
+
+
+def gather(cfg, st, sel, miss_count, ws, ws_bytes, stream=None):
+    _check(load().nosa_gather(ctypes.byref(cfg), ctypes.byref(st), _ptr(sel), _ptr(miss_count),
+                              _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def decode_attn(cfg, st, q, sel, out, ws, ws_bytes, stream=None):
+    _check(load().nosa_decode_attn(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(sel),
+                                   _ptr(out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def step(cfg, st, q, score_rows, k_new, v_new, evict, sel, out, miss_count, ws, ws_bytes,
+         stream=None, events: Optional[Sequence] = None):
+    ev = None
+    if events is not None:
+        ev = (ctypes.c_void_p * 4)(*[e.cuda_event if e is not None else None for e in events])
+    _check(load().nosa_step(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(score_rows),
+                            _ptr(k_new), _ptr(v_new), _ptr(evict), _ptr(sel), _ptr(out),
+                            _ptr(miss_count), _ptr(ws), ws_bytes, _stream(stream), ev))
+
+
+def check_device(st, stream=None):
+    """Synchronises; returns (status, error word) without raising."""
+    e = ctypes.c_uint32()
+    rc = load().nosa_check_device(ctypes.byref(st), _stream(stream), ctypes.byref(e))
+    return rc, e.value
+
+
+from .cache import NosaCache  # noqa: E402  (allocation helper on top of the ABI)

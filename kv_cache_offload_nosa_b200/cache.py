@@ -1,0 +1,79 @@
+"""Allocation helper: owns the decode-state buffers of one NOSA layer.
+
+Memory comes from PyTorch (device tensors, and pinned host tensors for the
+offloaded backing copy); all computation goes through the C ABI.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import (nosa_config, nosa_state, STATE_FIELDS, state_sizes, workspace_size, workspace_init,
+               state_init, append, score_blocks, select, gather, decode_attn, step, check_device)
+
+_DTYPE = {"seq_len": torch.int32, "kc": torch.float32, "prev_sel": torch.int32,
+          "alive": torch.int32, "last_used": torch.int32, "block_table": torch.int32,
+          "slot_owner": torch.int32, "k_pool": torch.int16, "v_pool": torch.int16,
+          "host_k": torch.int16, "host_v": torch.int16, "err": torch.int32}
+
+
+class NosaCache:
+    """Decode state + workspace for one configuration.
+
+    offload=True keeps the full K/V backing copy in pinned host memory and
+    `cfg.slots` pages per group in HBM; otherwise every block is in HBM.
+    """
+
+    def __init__(self, cfg: nosa_config, offload: bool = False, device: str = "cuda"):
+        self.cfg = cfg
+        self.offload = offload
+        self.device = torch.device(device)
+        sz = state_sizes(cfg)
+        self.t = {}
+        for name in STATE_FIELDS:
+            nbytes = getattr(sz, name)
+            dt = _DTYPE[name]
+            n = max(1, nbytes // torch.tensor([], dtype=dt).element_size())
+            if name in ("host_k", "host_v"):
+                self.t[name] = (torch.empty(n, dtype=dt, pin_memory=True) if offload else None)
+            else:
+                self.t[name] = torch.empty(n, dtype=dt, device=self.device)
+        self.ws_bytes = workspace_size(cfg)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        workspace_init(self.ws, self.ws_bytes)
+        self.state = nosa_state(*[(self.t[n].data_ptr() if self.t[n] is not None else None)
+                                  for n in STATE_FIELDS])
+
+    # views in the documented layouts
+    def pool_view(self, name: str) -> torch.Tensor:
+        c = self.cfg
+        G = c.B * c.Hkv
+        pages = c.max_blocks if name.startswith("host") else c.slots
+        return self.t[name].view(G, pages, c.block_size, c.d)
+
+    def init(self, prefill_len: torch.Tensor, resident: Optional[torch.Tensor] = None, stream=None):
+        state_init(self.cfg, self.state, prefill_len, resident, self.ws, self.ws_bytes, stream)
+
+    def append(self, k_new, v_new, stream=None):
+        append(self.cfg, self.state, k_new, v_new, stream)
+
+    def score_blocks(self, rows, block_scores, stream=None):
+        score_blocks(self.cfg, self.state, rows, block_scores, stream)
+
+    def select(self, block_scores, evict, sel, stream=None):
+        select(self.cfg, self.state, block_scores, evict, sel, stream)
+
+    def gather(self, sel, miss_count, stream=None):
+        gather(self.cfg, self.state, sel, miss_count, self.ws, self.ws_bytes, stream)
+
+    def decode_attn(self, q, sel, out, stream=None):
+        decode_attn(self.cfg, self.state, q, sel, out, self.ws, self.ws_bytes, stream)
+
+    def step(self, q, k_new, v_new, evict, sel, out, miss_count, score_rows=None, stream=None,
+             events=None):
+        step(self.cfg, self.state, q, score_rows, k_new, v_new, evict, sel, out, miss_count, self.ws,
+             self.ws_bytes, stream, events)
+
+    def check(self, stream=None):
+        return check_device(self.state, stream)

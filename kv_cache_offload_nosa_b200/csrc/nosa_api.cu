@@ -1,0 +1,541 @@
+// Host side of libnosa.so: argument validation, workspace layout, TMA
+// descriptors and kernel launches for the C ABI declared in include/nosa.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "nosa.h"
+#include "nosa_attn.cuh"
+#include "nosa_common.cuh"
+#include "nosa_kernels.cuh"
+#include "nosa_select.cuh"
+
+using namespace nosa;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+nosa_status fail(nosa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+#define NOSA_CHECK(cond, ...) \
+  do {                        \
+    if (!(cond)) return fail(NOSA_EINVAL, __VA_ARGS__); \
+  } while (0)
+
+#define NOSA_CUDA(call)                                                                    \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess) return fail(NOSA_ECUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int n_groups(const nosa_config& c) { return c.B * c.Hkv; }
+int max_sub(const nosa_config& c) { return c.max_blocks * (c.block_size / c.sub_block); }
+int words(const nosa_config& c) { return (c.max_blocks + 31) / 32; }
+int kk(const nosa_config& c) { return c.k_q + c.k_e; }
+
+nosa_status check_cfg(const nosa_config* cp) {
+  NOSA_CHECK(cp, "cfg is NULL");
+  const nosa_config& c = *cp;
+  NOSA_CHECK(c.B >= 1 && c.Hkv >= 1 && c.Hq >= c.Hkv && c.Hq % c.Hkv == 0,
+             "bad heads: B=%d Hq=%d Hkv=%d", c.B, c.Hq, c.Hkv);
+  const int G = c.Hq / c.Hkv;
+  NOSA_CHECK(G == 1 || G == 2 || G == 4 || G == 8, "G = Hq/Hkv = %d not in {1,2,4,8}", G);
+  NOSA_CHECK(c.d == 64 || c.d == 128, "d = %d not in {64,128}", c.d);
+  NOSA_CHECK(c.block_size == 32 || c.block_size == 64 || c.block_size == 128,
+             "block_size = %d not in {32,64,128}", c.block_size);
+  NOSA_CHECK((c.sub_block == 8 || c.sub_block == 16 || c.sub_block == 32) &&
+                 c.block_size % c.sub_block == 0,
+             "sub_block = %d must be 8, 16 or 32 and divide block_size", c.sub_block);
+  NOSA_CHECK(c.k_q >= 0 && c.k_e >= 0 && c.k_q + c.k_e >= 1, "bad budgets k_q=%d k_e=%d", c.k_q,
+             c.k_e);
+  NOSA_CHECK(c.max_blocks >= 1 && c.max_blocks <= kMaxBlocks, "max_blocks = %d not in [1, %d]",
+             c.max_blocks, kMaxBlocks);
+  NOSA_CHECK(kk(c) <= c.max_blocks, "k = %d > max_blocks = %d", kk(c), c.max_blocks);
+  NOSA_CHECK(c.slots >= 1 && c.slots <= c.max_blocks, "slots = %d not in [1, max_blocks]", c.slots);
+  NOSA_CHECK(c.n_score_rows == G || c.n_score_rows == 1, "n_score_rows = %d must be G or 1",
+             c.n_score_rows);
+  NOSA_CHECK(c.attn_split >= 0, "attn_split < 0");
+  NOSA_CHECK(c.scale > 0.f, "scale must be > 0");
+  const long long groups = (long long)c.B * c.Hkv;
+  NOSA_CHECK(groups * c.slots * c.block_size < (1ll << 31), "too many pool rows for TMA coordinates");
+  NOSA_CHECK(groups * kk(c) < (1ll << 31), "too many tasks");
+  return NOSA_OK;
+}
+
+bool has_host(const nosa_state* st) { return st->host_k != nullptr; }
+
+nosa_status check_state(const nosa_config& c, const nosa_state* st) {
+  NOSA_CHECK(st, "state is NULL");
+  const void* dev[] = {st->seq_len, st->kc, st->prev_sel, st->alive, st->last_used,
+                       st->block_table, st->slot_owner, st->k_pool, st->v_pool, st->err};
+  for (const void* p : dev) {
+    NOSA_CHECK(p, "a device state buffer is NULL");
+    NOSA_CHECK(aligned16(p), "state buffer %p not 16-byte aligned", p);
+  }
+  NOSA_CHECK((st->host_k == nullptr) == (st->host_v == nullptr), "host_k and host_v must both be set or both NULL");
+  if (has_host(st)) {
+    NOSA_CHECK(aligned16(st->host_k) && aligned16(st->host_v), "host pools not 16-byte aligned");
+    NOSA_CHECK(c.slots >= kk(c) + 2, "offload needs slots >= k + 2 (slots=%d, k=%d)", c.slots, kk(c));
+    for (const void* p : {(const void*)st->host_k, (const void*)st->host_v}) {
+      cudaPointerAttributes at;
+      cudaError_t e = cudaPointerGetAttributes(&at, p);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(NOSA_EINVAL, "host pool %p: %s", p, cudaGetErrorString(e));
+      }
+      NOSA_CHECK(at.type == cudaMemoryTypeHost && at.devicePointer == p,
+                 "host pool %p is not pinned, device-mapped host memory", p);
+    }
+  } else {
+    NOSA_CHECK(c.slots == c.max_blocks, "without host pools slots must equal max_blocks");
+  }
+  return NOSA_OK;
+}
+
+struct WsLayout {
+  size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, total;
+  int copy_stride;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(const nosa_config& c) {
+  WsLayout w;
+  const size_t NG = n_groups(c);
+  const int G = c.Hq / c.Hkv;
+  w.copy_stride = (kk(c) + 1 > c.slots) ? kk(c) + 1 : c.slots;
+  size_t off = 0;
+  w.scores = off; off += up256(NG * c.max_blocks * 4);
+  w.cnt_k1 = off; off += up256(NG * 4);
+  w.cnt_attn = off; off += up256(NG * 4);
+  w.copy_list = off; off += up256(NG * (size_t)w.copy_stride * 8);
+  w.copy_count = off; off += up256(NG * 4);
+  w.partials = off; off += up256(NG * kPartialSlots * (size_t)G * (c.d + 2) * 4);
+  w.total = off;
+  return w;
+}
+
+template <typename T>
+T* ws_at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+nosa_status check_ws(const nosa_config& c, void* ws, size_t bytes) {
+  NOSA_CHECK(ws && aligned16(ws), "workspace NULL or not 16-byte aligned");
+  const size_t need = ws_layout(c).total;
+  if (bytes < need) return fail(NOSA_ENOMEM, "workspace %zu bytes < %zu needed", bytes, need);
+  return NOSA_OK;
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+StepArgs step_args(const nosa_config& c, const nosa_state* st) {
+  StepArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kc = st->kc;
+  a.seq_len = st->seq_len;
+  a.max_blocks = c.max_blocks;
+  a.max_sub = max_sub(c);
+  a.bs = c.block_size;
+  a.s = c.sub_block;
+  a.slots = c.slots;
+  a.scale = c.scale;
+  a.total_pages = (long long)n_groups(c) * c.slots;
+  a.k_pool = st->k_pool;
+  a.v_pool = st->v_pool;
+  a.host_k = st->host_k;
+  a.host_v = st->host_v;
+  a.block_table = st->block_table;
+  a.prev_sel = st->prev_sel;
+  a.alive = st->alive;
+  a.k_q = c.k_q;
+  a.k_e = c.k_e;
+  a.slot_owner = st->slot_owner;
+  a.last_used = st->last_used;
+  a.err = st->err;
+  return a;
+}
+
+void set_ws(StepArgs& a, const nosa_config& c, void* ws) {
+  const WsLayout w = ws_layout(c);
+  a.copy_list = ws_at<int2>(ws, w.copy_list);
+  a.copy_stride = w.copy_stride;
+  a.copy_count = ws_at<int32_t>(ws, w.copy_count);
+  a.counters = ws_at<uint32_t>(ws, w.cnt_k1);
+}
+
+// ------------------------------------------------------------------ launches
+template <bool FUSED>
+nosa_status launch_score(const nosa_config& c, const StepArgs& a, cudaStream_t s) {
+  dim3 grid((max_sub(c) + kChunkSub - 1) / kChunkSub, n_groups(c));
+  const size_t dsm = FUSED ? sel_smem_bytes(c.max_blocks) : 0;
+  if (c.d == 128) {
+    auto k = score_kernel<128, FUSED>;
+    if (dsm > 48 * 1024) NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm));
+    k<<<grid, kScoreThreads, dsm, s>>>(a);
+  } else {
+    auto k = score_kernel<64, FUSED>;
+    if (dsm > 48 * 1024) NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm));
+    k<<<grid, kScoreThreads, dsm, s>>>(a);
+  }
+  NOSA_CUDA(cudaGetLastError());
+  return NOSA_OK;
+}
+
+nosa_status launch_sel_kernel(void (*k)(StepArgs), const nosa_config& c, const StepArgs& a,
+                              cudaStream_t s) {
+  const size_t dsm = sel_smem_bytes(c.max_blocks);
+  if (dsm > 48 * 1024)
+    NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm));
+  k<<<n_groups(c), kSelThreads, dsm, s>>>(a);
+  NOSA_CUDA(cudaGetLastError());
+  return NOSA_OK;
+}
+
+nosa_status launch_copy(const nosa_config& c, const nosa_state* st, void* ws, cudaStream_t s) {
+  const WsLayout w = ws_layout(c);
+  const int page_vec = c.block_size * c.d * 2 / 16;
+  dim3 grid(n_groups(c), 8);
+  copy_kernel<<<grid, 256, 0, s>>>(ws_at<int2>(ws, w.copy_list), w.copy_stride,
+                                   ws_at<int32_t>(ws, w.copy_count),
+                                   reinterpret_cast<const uint4*>(st->host_k),
+                                   reinterpret_cast<const uint4*>(st->host_v),
+                                   reinterpret_cast<uint4*>(st->k_pool),
+                                   reinterpret_cast<uint4*>(st->v_pool), c.max_blocks, page_vec);
+  NOSA_CUDA(cudaGetLastError());
+  return NOSA_OK;
+}
+
+// ---- TMA descriptors (driver entry point fetched through the runtime; no -lcuda)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+nosa_status get_encode(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  if (!cached) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    NOSA_CUDA(cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q));
+    if (q != cudaDriverEntryPointSuccess || !p) return fail(NOSA_ECUDA, "cuTensorMapEncodeTiled unavailable");
+    cached = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *fn = cached;
+  return NOSA_OK;
+}
+
+nosa_status make_pool_map(CUtensorMap* m, const nosa_config& c, void* pool) {
+  EncodeTiledFn enc;
+  nosa_status r = get_encode(&enc);
+  if (r != NOSA_OK) return r;
+  const cuuint64_t rows = (cuuint64_t)n_groups(c) * c.slots * c.block_size;
+  cuuint64_t dims[2] = {(cuuint64_t)c.d, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)c.d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)c.block_size};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult e = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pool, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (e != CUDA_SUCCESS) return fail(NOSA_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)e);
+  return NOSA_OK;
+}
+
+template <int D, int BS>
+nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& tk, const CUtensorMap& tv,
+                          cudaStream_t s) {
+  using SH = AttnShape<D, BS>;
+  int stages = (110 * 1024) / SH::STAGE;
+  stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
+  const size_t smem = SH::smem_bytes(stages);
+  auto k = attn_kernel<D, BS>;
+  NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int dev = 0, sms = 0, per_sm = 0;
+  NOSA_CUDA(cudaGetDevice(&dev));
+  NOSA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  NOSA_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, SH::THREADS, smem));
+  if (per_sm < 1) per_sm = 1;
+  const long long target = (long long)sms * per_sm;
+  int W = c.attn_split > 0 ? c.attn_split : (int)((a.total + target - 1) / target);
+  const int wmin = (a.k + kPartialSlots - 2) / (kPartialSlots - 1);
+  if (W < wmin) W = wmin;
+  if (W < 1) W = 1;
+  a.W = W;
+  a.stages = stages;
+  const int grid = (a.total + W - 1) / W;
+  k<<<grid, SH::THREADS, smem, s>>>(tk, tv, a);
+  NOSA_CUDA(cudaGetLastError());
+  return NOSA_OK;
+}
+
+nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16_t* q, const int32_t* sel,
+                        float* out, void* ws, cudaStream_t s) {
+  CUtensorMap tk, tv;
+  nosa_status r = make_pool_map(&tk, c, st->k_pool);
+  if (r != NOSA_OK) return r;
+  r = make_pool_map(&tv, c, st->v_pool);
+  if (r != NOSA_OK) return r;
+  const WsLayout w = ws_layout(c);
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = q;
+  a.sel = sel;
+  a.seq_len = st->seq_len;
+  a.block_table = st->block_table;
+  a.out = out;
+  a.partials = ws_at<float>(ws, w.partials);
+  a.counters = ws_at<uint32_t>(ws, w.cnt_attn);
+  a.err = st->err;
+  a.Hq = c.Hq;
+  a.Hkv = c.Hkv;
+  a.G = c.Hq / c.Hkv;
+  a.k = kk(c);
+  a.max_blocks = c.max_blocks;
+  a.total = n_groups(c) * kk(c);
+  a.total_pages = (long long)n_groups(c) * c.slots;
+  a.scale_log2 = c.scale * 1.4426950408889634f;
+  if (c.d == 128) {
+    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s);
+    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s);
+    return launch_attn_t<128, 128>(c, a, tk, tv, s);
+  }
+  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s);
+  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s);
+  return launch_attn_t<64, 128>(c, a, tk, tv, s);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* nosa_status_string(nosa_status s) {
+  switch (s) {
+    case NOSA_OK: return "ok";
+    case NOSA_EINVAL: return "invalid argument";
+    case NOSA_ENOMEM: return "workspace too small";
+    case NOSA_ECUDA: return "CUDA runtime error";
+    case NOSA_EDEVICE: return "device-side fault recorded";
+    case NOSA_ETIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* nosa_last_error(void) { return g_err; }
+
+nosa_status nosa_state_sizes(const nosa_config* cfg, nosa_sizes* out) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  NOSA_CHECK(out, "out is NULL");
+  const nosa_config& c = *cfg;
+  const size_t NG = n_groups(c);
+  out->seq_len = NG * 4;
+  out->kc = NG * max_sub(c) * (size_t)c.d * 4;
+  out->prev_sel = NG * words(c) * 4;
+  out->alive = NG * words(c) * 4;
+  out->last_used = NG * c.max_blocks * 4;
+  out->block_table = NG * c.max_blocks * 4;
+  out->slot_owner = NG * c.slots * 4;
+  out->k_pool = NG * c.slots * (size_t)c.block_size * c.d * 2;
+  out->v_pool = out->k_pool;
+  out->host_k = NG * c.max_blocks * (size_t)c.block_size * c.d * 2;
+  out->host_v = out->host_k;
+  out->err = 4;
+  return NOSA_OK;
+}
+
+nosa_status nosa_workspace_size(const nosa_config* cfg, size_t* bytes) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  NOSA_CHECK(bytes, "bytes is NULL");
+  *bytes = ws_layout(*cfg).total;
+  return NOSA_OK;
+}
+
+nosa_status nosa_workspace_init(void* ws, size_t bytes, void* stream) {
+  NOSA_CHECK(ws && aligned16(ws), "workspace NULL or not 16-byte aligned");
+  NOSA_CUDA(cudaMemsetAsync(ws, 0, bytes, as_stream(stream)));
+  return NOSA_OK;
+}
+
+nosa_status nosa_state_init(const nosa_config* cfg, const nosa_state* st, const int32_t* prefill_len,
+                            const uint8_t* resident, void* ws, size_t ws_bytes, void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
+  NOSA_CHECK(prefill_len, "prefill_len is NULL");
+  cudaStream_t s = as_stream(stream);
+  NOSA_CUDA(cudaMemsetAsync(st->err, 0, 4, s));
+  const WsLayout w = ws_layout(c);
+  InitArgs a;
+  a.prefill_len = prefill_len;
+  a.resident = resident;
+  a.seq_len = st->seq_len;
+  a.prev_sel = st->prev_sel;
+  a.alive = st->alive;
+  a.last_used = st->last_used;
+  a.block_table = st->block_table;
+  a.slot_owner = st->slot_owner;
+  a.copy_list = ws_at<int2>(ws, w.copy_list);
+  a.copy_stride = w.copy_stride;
+  a.copy_count = ws_at<int32_t>(ws, w.copy_count);
+  a.err = st->err;
+  a.Hkv = c.Hkv;
+  a.bs = c.block_size;
+  a.max_blocks = c.max_blocks;
+  a.slots = c.slots;
+  a.host = has_host(st) ? 1 : 0;
+  init_tables_kernel<<<n_groups(c), 256, 0, s>>>(a);
+  NOSA_CUDA(cudaGetLastError());
+  const uint16_t* src = has_host(st) ? st->host_k : st->k_pool;
+  const int ppg = has_host(st) ? c.max_blocks : c.slots;
+  const int subs = 256 / c.d * 4;
+  dim3 g((max_sub(c) + subs - 1) / subs, n_groups(c));
+  if (c.d == 128)
+    init_kc_kernel<128><<<g, 256, 0, s>>>(prefill_len, c.Hkv, src, ppg, st->kc, max_sub(c), c.block_size, c.sub_block);
+  else
+    init_kc_kernel<64><<<g, 256, 0, s>>>(prefill_len, c.Hkv, src, ppg, st->kc, max_sub(c), c.block_size, c.sub_block);
+  NOSA_CUDA(cudaGetLastError());
+  if (has_host(st)) return launch_copy(c, st, ws, s);
+  return NOSA_OK;
+}
+
+nosa_status nosa_append(const nosa_config* cfg, const nosa_state* st, const uint16_t* k_new,
+                        const uint16_t* v_new, void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  NOSA_CHECK(k_new && v_new && aligned16(k_new) && aligned16(v_new), "k_new/v_new NULL or misaligned");
+  StepArgs a = step_args(c, st);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  if (c.d == 128) append_kernel<128><<<n_groups(c), 128, 0, as_stream(stream)>>>(a);
+  else append_kernel<64><<<n_groups(c), 128, 0, as_stream(stream)>>>(a);
+  NOSA_CUDA(cudaGetLastError());
+  return NOSA_OK;
+}
+
+nosa_status nosa_score_blocks(const nosa_config* cfg, const nosa_state* st, const uint16_t* rows,
+                              float* block_scores, void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  NOSA_CHECK(rows && block_scores && aligned16(rows) && aligned16(block_scores),
+             "score rows / block_scores NULL or misaligned");
+  StepArgs a = step_args(c, st);
+  a.rows = rows;
+  a.R = c.n_score_rows;
+  a.block_scores = block_scores;
+  return launch_score<false>(c, a, as_stream(stream));
+}
+
+nosa_status nosa_select(const nosa_config* cfg, const nosa_state* st, const float* block_scores,
+                        const float* evict, int32_t* sel, void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  NOSA_CHECK(block_scores && evict && sel && aligned16(block_scores) && aligned16(evict) && aligned16(sel),
+             "select buffers NULL or misaligned");
+  StepArgs a = step_args(c, st);
+  a.block_scores = const_cast<float*>(block_scores);
+  a.evict = evict;
+  a.sel = sel;
+  return launch_sel_kernel(select_kernel, c, a, as_stream(stream));
+}
+
+nosa_status nosa_gather(const nosa_config* cfg, const nosa_state* st, const int32_t* sel,
+                        int32_t* miss_count, void* ws, size_t ws_bytes, void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
+  NOSA_CHECK(sel && miss_count && aligned16(sel) && aligned16(miss_count), "sel/miss_count NULL or misaligned");
+  cudaStream_t s = as_stream(stream);
+  if (!has_host(st)) {
+    NOSA_CUDA(cudaMemsetAsync(miss_count, 0, (size_t)n_groups(c) * 4, s));
+    return NOSA_OK;
+  }
+  StepArgs a = step_args(c, st);
+  set_ws(a, c, ws);
+  a.sel = const_cast<int32_t*>(sel);
+  a.miss_count = miss_count;
+  if ((r = launch_sel_kernel(plan_kernel, c, a, s)) != NOSA_OK) return r;
+  return launch_copy(c, st, ws, s);
+}
+
+nosa_status nosa_decode_attn(const nosa_config* cfg, const nosa_state* st, const uint16_t* q,
+                             const int32_t* sel, float* out, void* ws, size_t ws_bytes, void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
+  NOSA_CHECK(q && sel && out && aligned16(q) && aligned16(sel) && aligned16(out), "q/sel/out NULL or misaligned");
+  return launch_attn(c, st, q, sel, out, ws, as_stream(stream));
+}
+
+nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16_t* q,
+                      const uint16_t* score_rows, const uint16_t* k_new, const uint16_t* v_new,
+                      const float* evict, int32_t* sel, float* out, int32_t* miss_count, void* ws,
+                      size_t ws_bytes, void* stream, void* const* events) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
+  NOSA_CHECK(q && k_new && v_new && evict && sel && out && miss_count, "step buffer is NULL");
+  const void* ptrs[] = {q, k_new, v_new, evict, sel, out, miss_count};
+  for (const void* p : ptrs) NOSA_CHECK(aligned16(p), "step buffer %p not 16-byte aligned", p);
+  NOSA_CHECK(score_rows || c.n_score_rows == c.Hq / c.Hkv, "score_rows NULL requires n_score_rows == G");
+  NOSA_CHECK(!score_rows || aligned16(score_rows), "score_rows misaligned");
+  cudaStream_t s = as_stream(stream);
+  auto rec = [&](int i) -> nosa_status {
+    if (events && events[i]) NOSA_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s));
+    return NOSA_OK;
+  };
+  if ((r = rec(0)) != NOSA_OK) return r;
+  StepArgs a = step_args(c, st);
+  set_ws(a, c, ws);
+  a.rows = score_rows ? score_rows : q;
+  a.R = c.n_score_rows;
+  a.block_scores = ws_at<float>(ws, ws_layout(c).scores);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.evict = evict;
+  a.sel = sel;
+  a.miss_count = miss_count;
+  if ((r = launch_score<true>(c, a, s)) != NOSA_OK) return r;
+  if ((r = rec(1)) != NOSA_OK) return r;
+  if (has_host(st) && (r = launch_copy(c, st, ws, s)) != NOSA_OK) return r;
+  if ((r = rec(2)) != NOSA_OK) return r;
+  if ((r = launch_attn(c, st, q, sel, out, ws, s)) != NOSA_OK) return r;
+  return rec(3);
+}
+
+nosa_status nosa_check_device(const nosa_state* st, void* stream, uint32_t* err_out) {
+  NOSA_CHECK(st && st->err, "state/err is NULL");
+  uint32_t e = 0;
+  NOSA_CUDA(cudaMemcpyAsync(&e, st->err, 4, cudaMemcpyDeviceToHost, as_stream(stream)));
+  NOSA_CUDA(cudaStreamSynchronize(as_stream(stream)));
+  if (err_out) *err_out = e;
+  if (e & NOSA_ERR_TIMEOUT) return fail(NOSA_ETIMEOUT, "device wait timed out (err=0x%x)", e);
+  if (e) return fail(NOSA_EDEVICE, "device fault bits 0x%x", e);
+  return NOSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,399 @@
+// Score / append / select / gather / init kernels of the NOSA decode step.
+//
+// score_kernel streams the fp32 sub-block mean keys (kc) of every group once:
+// HBM-bound at one FMA per 4 bytes, so it is written for coalesced 16-byte
+// loads (each warp covers whole sub-blocks with 128-byte segments), a grid of
+// B*Hkv x ceil(max_sub/256) CTAs of 256 threads, and warp-shuffle reductions.
+// Fused form: the CTA owning the tail sub-block appends the new token first,
+// and the last CTA of each group to finish (atomic ticket, no spinning) runs
+// the dual selection and, with host pools, the residency plan.
+#pragma once
+
+#include "nosa_select.cuh"
+
+namespace nosa {
+
+constexpr int kScoreThreads = 256;
+constexpr int kChunkSub = 256;  // sub-blocks per score CTA
+
+struct StepArgs {
+  // scoring
+  const uint16_t* rows;   // [B*Hkv][R][d] bf16
+  int R;
+  float* kc;
+  float* block_scores;    // [B*Hkv][max_blocks]
+  int32_t* seq_len;
+  int max_blocks, max_sub, bs, s, slots;
+  float scale;
+  long long total_pages;
+  // append
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint16_t* k_pool;
+  uint16_t* v_pool;
+  uint16_t* host_k;
+  uint16_t* host_v;
+  int32_t* block_table;
+  // selection
+  const float* evict;
+  uint32_t* prev_sel;
+  uint32_t* alive;
+  int32_t* sel;
+  int k_q, k_e;
+  // residency
+  int32_t* slot_owner;
+  int32_t* last_used;
+  int2* copy_list;
+  int copy_stride;
+  int32_t* copy_count;
+  int32_t* miss_count;
+  uint32_t* counters;
+  uint32_t* err;
+};
+
+// Append token pos = len0 of group gi (all threads of the CTA take part).
+template <int D>
+__device__ void append_token(const StepArgs& a, int gi, int len0) {
+  const int pos = len0;
+  const int jb = pos / a.bs, r = pos % a.bs, sb = pos / a.s;
+  int page = a.block_table[(size_t)gi * a.max_blocks + jb];
+  if (page >= a.total_pages || (page < 0 && !a.host_k)) {
+    if (threadIdx.x == 0) set_err(a.err, NOSA_ERR_BLOCK_TABLE);
+    page = -1;
+  }
+  const size_t hbase = ((size_t)gi * a.max_blocks + jb) * a.bs;
+  const int t0 = sb * a.s;
+  for (int x = threadIdx.x; x < D; x += blockDim.x) {
+    const uint16_t kx = a.k_new[(size_t)gi * D + x];
+    const uint16_t vx = a.v_new[(size_t)gi * D + x];
+    float sum = 0.f;
+    if (page >= 0 || a.host_k) {
+      for (int tau = t0; tau < pos; ++tau) {
+        const int rr = tau - jb * a.bs;
+        const uint16_t* src = (page >= 0) ? a.k_pool + ((size_t)page * a.bs + rr) * D
+                                          : a.host_k + (hbase + rr) * D;
+        sum += bf16_bits_to_f32(src[x]);
+      }
+    }
+    sum += bf16_bits_to_f32(kx);
+    if (page >= 0) {
+      a.k_pool[((size_t)page * a.bs + r) * D + x] = kx;
+      a.v_pool[((size_t)page * a.bs + r) * D + x] = vx;
+    }
+    if (a.host_k) {
+      a.host_k[(hbase + r) * D + x] = kx;
+      a.host_v[(hbase + r) * D + x] = vx;
+    }
+    a.kc[((size_t)gi * a.max_sub + sb) * D + x] = __fdiv_rn(sum, (float)(pos - t0 + 1));
+  }
+}
+
+template <int D, bool FUSED>
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
+  constexpr int LPS = D / 16;        // lanes per sub-block (16 floats each)
+  constexpr int SPW = 32 / LPS;      // sub-blocks per warp pass
+  constexpr int PASS = SPW * (kScoreThreads / 32);
+  __shared__ float qbar[D];
+  __shared__ float su[kChunkSub];
+  __shared__ int s_last;
+  extern __shared__ __align__(16) uint8_t dsm[];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gi = blockIdx.y, c = blockIdx.x;
+  const int len0 = a.seq_len[gi];
+  int L = len0;
+  if (FUSED) {
+    if (len0 < a.max_blocks * a.bs) L = len0 + 1;
+    else if (c == 0 && tid == 0) set_err(a.err, NOSA_ERR_FULL);
+  }
+  const int M = (L + a.s - 1) / a.s;
+  const int N = (L + a.bs - 1) / a.bs;
+  const int spb = a.bs / a.s;
+  const int i0 = c * kChunkSub;
+  const int i1 = min(i0 + kChunkSub, M);
+
+  if (FUSED && L > len0 && (len0 / a.s) / kChunkSub == c) {
+    append_token<D>(a, gi, len0);
+    __syncthreads();
+  }
+  for (int x = tid; x < D; x += kScoreThreads) {
+    const uint16_t* r = a.rows + (size_t)gi * a.R * D + x;
+    float sacc = 0.f;
+    for (int rr = 0; rr < a.R; ++rr) sacc += bf16_bits_to_f32(r[(size_t)rr * D]);
+    qbar[x] = a.scale * sacc / (float)a.R;
+  }
+  __syncthreads();
+
+  if (i0 < i1) {
+    const int sub = lane / LPS, part = lane % LPS;
+    float qr[16];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int p4 = part + LPS * jj;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qr[4 * jj + e] = qbar[4 * p4 + e];
+    }
+    const float4* kcg = reinterpret_cast<const float4*>(a.kc + (size_t)gi * a.max_sub * D);
+    for (int base = i0 + warp * SPW; base < i1; base += 2 * PASS) {
+      const int ia = base + sub, ib = base + PASS + sub;
+      float4 va[4], vb[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int p4 = part + LPS * jj;
+        va[jj] = (ia < i1) ? __ldcs(kcg + (size_t)ia * (D / 4) + p4) : make_float4(0, 0, 0, 0);
+        vb[jj] = (ib < i1) ? __ldcs(kcg + (size_t)ib * (D / 4) + p4) : make_float4(0, 0, 0, 0);
+      }
+      float da = 0.f, db = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        da = fmaf(qr[4 * jj + 0], va[jj].x, da);
+        da = fmaf(qr[4 * jj + 1], va[jj].y, da);
+        da = fmaf(qr[4 * jj + 2], va[jj].z, da);
+        da = fmaf(qr[4 * jj + 3], va[jj].w, da);
+        db = fmaf(qr[4 * jj + 0], vb[jj].x, db);
+        db = fmaf(qr[4 * jj + 1], vb[jj].y, db);
+        db = fmaf(qr[4 * jj + 2], vb[jj].z, db);
+        db = fmaf(qr[4 * jj + 3], vb[jj].w, db);
+      }
+#pragma unroll
+      for (int o = LPS / 2; o >= 1; o >>= 1) {
+        da += __shfl_xor_sync(0xffffffffu, da, o);
+        db += __shfl_xor_sync(0xffffffffu, db, o);
+      }
+      if (part == 0) {
+        if (ia < i1) su[ia - i0] = da;
+        if (ib < i1) su[ib - i0] = db;
+      }
+    }
+  }
+  __syncthreads();
+  // block max over present sub-blocks; -inf for blocks not yet created
+  {
+    const int j = i0 / spb + tid;
+    if (tid < kChunkSub / spb && j < a.max_blocks) {
+      float m = -INFINITY;
+      if (j < N) {
+        const int e = min((j + 1) * spb, M);
+        for (int i = j * spb; i < e; ++i) m = fmaxf(m, su[i - i0]);
+      }
+      a.block_scores[(size_t)gi * a.max_blocks + j] = m;
+    }
+  }
+  if (!FUSED) return;
+
+  // last chunk of this group to finish runs the selection
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&a.counters[gi], 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const SelSmem S = sel_smem_carve(dsm, a.max_blocks);
+  const int Wmax = (a.max_blocks + 31) / 32;
+  const int k = a.k_q + a.k_e;
+  select_group(S, a.block_scores + (size_t)gi * a.max_blocks, a.evict + (size_t)gi * a.max_blocks,
+               a.prev_sel + (size_t)gi * Wmax, a.alive + (size_t)gi * Wmax, a.sel + (size_t)gi * k,
+               N, a.k_e, k, Wmax);
+  if (a.host_k) {
+    PlanArgs p;
+    p.block_table = a.block_table + (size_t)gi * a.max_blocks;
+    p.slot_owner = a.slot_owner + (size_t)gi * a.slots;
+    p.last_used = a.last_used + (size_t)gi * a.max_blocks;
+    p.copy_list = a.copy_list + (size_t)gi * a.copy_stride;
+    p.copy_count = a.copy_count + gi;
+    p.miss_count = a.miss_count ? a.miss_count + gi : nullptr;
+    p.err = a.err;
+    p.L = L;
+    p.bs = a.bs;
+    p.slots = a.slots;
+    p.page_base = gi * a.slots;
+    p.max_blocks = a.max_blocks;
+    plan_group(S, p);
+  } else if (a.miss_count && tid == 0) {
+    a.miss_count[gi] = 0;
+  }
+  if (tid == 0) {
+    a.counters[gi] = 0u;
+    a.seq_len[gi] = L;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) append_kernel(StepArgs a) {
+  const int gi = blockIdx.x;
+  const int len0 = a.seq_len[gi];
+  if (len0 >= a.max_blocks * a.bs) {
+    if (threadIdx.x == 0) set_err(a.err, NOSA_ERR_FULL);
+    return;
+  }
+  append_token<D>(a, gi, len0);
+  __syncthreads();
+  if (threadIdx.x == 0) a.seq_len[gi] = len0 + 1;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(StepArgs a) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const int gi = blockIdx.x;
+  const int L = a.seq_len[gi];
+  const int N = (L + a.bs - 1) / a.bs;
+  const SelSmem S = sel_smem_carve(dsm, a.max_blocks);
+  const int Wmax = (a.max_blocks + 31) / 32;
+  const int k = a.k_q + a.k_e;
+  select_group(S, a.block_scores + (size_t)gi * a.max_blocks, a.evict + (size_t)gi * a.max_blocks,
+               a.prev_sel + (size_t)gi * Wmax, a.alive + (size_t)gi * Wmax, a.sel + (size_t)gi * k,
+               N, a.k_e, k, Wmax);
+}
+
+__global__ void __launch_bounds__(kSelThreads) plan_kernel(StepArgs a) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const int gi = blockIdx.x;
+  const int L = a.seq_len[gi];
+  const int N = (L + a.bs - 1) / a.bs;
+  const SelSmem S = sel_smem_carve(dsm, a.max_blocks);
+  const int Wmax = (a.max_blocks + 31) / 32;
+  const int k = a.k_q + a.k_e;
+  sset_from_list(S, a.sel + (size_t)gi * k, k, N, Wmax, a.err);
+  PlanArgs p;
+  p.block_table = a.block_table + (size_t)gi * a.max_blocks;
+  p.slot_owner = a.slot_owner + (size_t)gi * a.slots;
+  p.last_used = a.last_used + (size_t)gi * a.max_blocks;
+  p.copy_list = a.copy_list + (size_t)gi * a.copy_stride;
+  p.copy_count = a.copy_count + gi;
+  p.miss_count = a.miss_count ? a.miss_count + gi : nullptr;
+  p.err = a.err;
+  p.L = L;
+  p.bs = a.bs;
+  p.slots = a.slots;
+  p.page_base = gi * a.slots;
+  p.max_blocks = a.max_blocks;
+  plan_group(S, p);
+}
+
+// Host -> HBM page copies over UVA (pinned host memory read by the kernel with 16-byte
+// loads; NOSA's "Comunicacion de Alto Ancho de Banda"). grid = (groups, CTAs per group).
+__global__ void __launch_bounds__(256) copy_kernel(const int2* copy_list, int copy_stride,
+                                                   const int32_t* copy_count, const uint4* host_k,
+                                                   const uint4* host_v, uint4* k_pool, uint4* v_pool,
+                                                   int max_blocks, int page_vec) {
+  const int gi = blockIdx.x;
+  const int n = copy_count[gi];
+  for (int i = blockIdx.y; i < n; i += gridDim.y) {
+    const int2 e = copy_list[(size_t)gi * copy_stride + i];
+    const size_t src = ((size_t)gi * max_blocks + e.x) * page_vec;
+    const size_t dst = (size_t)e.y * page_vec;
+    for (int v0 = threadIdx.x; v0 < page_vec; v0 += 4 * blockDim.x) {
+      uint4 rk[4], rv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * blockDim.x;
+        if (v < page_vec) {
+          rk[u] = host_k[src + v];
+          rv[u] = host_v[src + v];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * blockDim.x;
+        if (v < page_vec) {
+          k_pool[dst + v] = rk[u];
+          v_pool[dst + v] = rv[u];
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ state init
+struct InitArgs {
+  const int32_t* prefill_len;
+  const uint8_t* resident;
+  int32_t* seq_len;
+  uint32_t* prev_sel;
+  uint32_t* alive;
+  int32_t* last_used;
+  int32_t* block_table;
+  int32_t* slot_owner;
+  int2* copy_list;
+  int copy_stride;
+  int32_t* copy_count;
+  uint32_t* err;
+  int Hkv, bs, max_blocks, slots, host;
+};
+
+__global__ void __launch_bounds__(256) init_tables_kernel(InitArgs a) {
+  __shared__ int red[33];
+  const int gi = blockIdx.x, tid = threadIdx.x;
+  const int T = a.prefill_len[gi / a.Hkv];
+  const int n0 = (T + a.bs - 1) / a.bs;
+  const int Wmax = (a.max_blocks + 31) / 32;
+  if (tid == 0) a.seq_len[gi] = T;
+  for (int w = tid; w < Wmax; w += blockDim.x) {
+    a.prev_sel[(size_t)gi * Wmax + w] = word_valid_mask(w, n0);
+    a.alive[(size_t)gi * Wmax + w] = word_valid_mask(w, a.max_blocks);
+  }
+  for (int j = tid; j < a.max_blocks; j += blockDim.x) a.last_used[(size_t)gi * a.max_blocks + j] = 0;
+  int32_t* bt = a.block_table + (size_t)gi * a.max_blocks;
+  int32_t* so = a.slot_owner + (size_t)gi * a.slots;
+  if (!a.host) {
+    for (int j = tid; j < a.max_blocks; j += blockDim.x) {
+      bt[j] = gi * a.slots + j;
+      so[j] = j;
+    }
+    if (tid == 0) a.copy_count[gi] = 0;
+    return;
+  }
+  // resident blocks take slots 0, 1, ... in ascending block order
+  const uint8_t* rf = a.resident ? a.resident + (size_t)gi * a.max_blocks : nullptr;
+  uint32_t m = 0;
+  if (tid < Wmax && rf) {
+    for (int b = 0; b < 32; ++b) {
+      const int j = tid * 32 + b;
+      if (j < a.max_blocks && rf[j]) m |= 1u << b;
+    }
+  }
+  int total;
+  const int before = block_exclusive_scan(__popc(m), red, &total);
+  if (total > a.slots && tid == 0) set_err(a.err, NOSA_ERR_INIT);
+  for (int j = tid; j < a.max_blocks; j += blockDim.x) bt[j] = -1;
+  for (int z = tid; z < a.slots; z += blockDim.x) so[z] = -1;
+  __syncthreads();
+  if (tid < Wmax) {
+    uint32_t t = m;
+    int r = before;
+    while (t) {
+      const int b = __ffs(t) - 1;
+      t &= t - 1;
+      if (r < a.slots) {
+        const int j = tid * 32 + b;
+        bt[j] = gi * a.slots + r;
+        so[r] = j;
+        a.copy_list[(size_t)gi * a.copy_stride + r] = make_int2(j, gi * a.slots + r);
+      }
+      ++r;
+    }
+  }
+  if (tid == 0) a.copy_count[gi] = total < a.slots ? total : a.slots;
+}
+
+// kc[i] = fp32 mean of the present tokens of sub-block i (prefill), zero past the prefill.
+template <int D>
+__global__ void __launch_bounds__(256) init_kc_kernel(const int32_t* prefill_len, int Hkv,
+                                                      const uint16_t* src, int src_pages_per_group,
+                                                      float* kc, int max_sub, int bs, int s) {
+  const int gi = blockIdx.y;
+  const int T = prefill_len[gi / Hkv];
+  constexpr int SUBS = 256 / D * 4;  // sub-blocks per CTA pass
+  for (int e = threadIdx.x; e < SUBS * D; e += blockDim.x) {
+    const int i = blockIdx.x * SUBS + e / D, x = e % D;
+    if (i >= max_sub) continue;
+    const int t0 = i * s, t1 = min(t0 + s, T);
+    float sum = 0.f;
+    for (int tau = t0; tau < t1; ++tau) {
+      const int j = tau / bs, r = tau % bs;
+      sum += bf16_bits_to_f32(src[(((size_t)gi * src_pages_per_group + j) * bs + r) * D + x]);
+    }
+    kc[((size_t)gi * max_sub + i) * D + x] = (t1 > t0) ? __fdiv_rn(sum, (float)(t1 - t0)) : 0.f;
+  }
+}
+
+}  // namespace nosa

@@ -71,9 +71,9 @@ def load(path: Optional[str] = None):
         L.orc_init.restype = ctypes.c_int
         L.orc_append.argtypes = [vp, vp, vp, vp]
         L.orc_append.restype = None
-        L.orc_block_scores.argtypes = [vp, vp, vp, vp]
+        L.orc_block_scores.argtypes = [vp, vp, vp, vp, vp]
         L.orc_block_scores.restype = None
-        L.orc_select.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_int]
+        L.orc_select.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
         L.orc_select.restype = None
         L.orc_residency.argtypes = [vp, vp, vp, vp]
         L.orc_residency.restype = ctypes.c_int
@@ -102,15 +102,19 @@ class Oracle:
     """Oracle state for one configuration, advanced step by step."""
 
     def __init__(self, cfg: syn.NosaConfig, pool_k: np.ndarray, pool_v: np.ndarray,
-                 resident: Optional[np.ndarray] = None, lib_path: Optional[str] = None):
+                 resident: Optional[np.ndarray] = None, lib_path: Optional[str] = None,
+                 copy: bool = True):
         self.cfg = cfg
         self.L = load(lib_path)
         c = cfg
         NG, nb = c.B * c.Hkv, c.max_blocks
         self.c = OrcCfg(c.B, c.Hq, c.Hkv, c.d, c.block, c.sub_block, c.k_q, c.k_e, c.rows, nb,
                         c.n_slots, int(c.offload), c.scale)
-        self.K = np.ascontiguousarray(pool_k).copy()
-        self.V = np.ascontiguousarray(pool_v).copy()
+        # copy=False: the oracle appends into the caller's arrays (rows >= T change)
+        self.K = np.ascontiguousarray(pool_k)
+        self.V = np.ascontiguousarray(pool_v)
+        if copy:
+            self.K, self.V = self.K.copy(), self.V.copy()
         self.kbar = np.zeros((NG, c.max_sub, c.d), np.float64)
         self.len = np.zeros(NG, np.int32)
         self.prev_sel = np.zeros((NG, nb), np.uint8)
@@ -131,23 +135,27 @@ class Oracle:
         self.L.orc_append(ctypes.byref(self.c), ctypes.byref(self.st),
                           _p(np.ascontiguousarray(k_new)), _p(np.ascontiguousarray(v_new)))
 
-    def block_scores(self, rows: np.ndarray) -> np.ndarray:
+    def block_scores(self, rows: np.ndarray, out: Optional[np.ndarray] = None,
+                     gmask: Optional[np.ndarray] = None) -> np.ndarray:
         c = self.cfg
-        out = np.empty((c.B * c.Hkv, c.max_blocks), np.float64)
+        if out is None:
+            out = np.empty((c.B * c.Hkv, c.max_blocks), np.float64)
+        gm = None if gmask is None else np.ascontiguousarray(gmask, np.uint8)
         self.L.orc_block_scores(ctypes.byref(self.c), ctypes.byref(self.st),
-                                _p(np.ascontiguousarray(rows)), _p(out))
+                                _p(np.ascontiguousarray(rows)), _p(out), _p(gm))
         return out
 
-    def select(self, scores, evict, commit=True):
+    def select(self, scores, evict, commit=True, gmask=None, out=None):
         c = self.cfg
         NG = c.B * c.Hkv
-        sel = np.empty((NG, c.k), np.int32)
-        src = np.empty((NG, c.k), np.int8)
-        gap = np.empty(NG, np.float64)
+        sel, src, gap = out if out is not None else (np.empty((NG, c.k), np.int32),
+                                                      np.empty((NG, c.k), np.int8),
+                                                      np.empty(NG, np.float64))
+        gm = None if gmask is None else np.ascontiguousarray(gmask, np.uint8)
         self.L.orc_select(ctypes.byref(self.c), ctypes.byref(self.st),
                           _p(np.ascontiguousarray(scores, np.float64)),
                           _p(np.ascontiguousarray(evict, np.float32)), _p(sel), _p(src), _p(gap),
-                          int(commit))
+                          int(commit), _p(gm))
         return sel, src, gap
 
     def residency(self, sel):
@@ -204,7 +212,8 @@ def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = M
     recorded, so the GPU and the oracle consume identical arrays.
     """
     inp = syn.make_inputs(cfg)
-    orc = Oracle(cfg, inp.pool_k, inp.pool_v, inp.resident, lib_path)
+    # the oracle appends in place: inp.pool_k / pool_v rows >= T then hold the decode tokens
+    orc = Oracle(cfg, inp.pool_k, inp.pool_v, inp.resident, lib_path, copy=False)
     S = cfg.steps if steps is None else steps
     G, R = cfg.G, cfg.rows
     prev = None
@@ -212,7 +221,10 @@ def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = M
     for t in range(S):
         orc.append(inp.k_new[t], inp.v_new[t])
         retry = np.zeros((cfg.B, cfg.Hkv), np.int64)
-        pending = np.ones((cfg.B, cfg.Hkv), bool)
+        todo = np.ones(cfg.B * cfg.Hkv, np.uint8)
+        scores = np.empty((cfg.B * cfg.Hkv, cfg.max_blocks), np.float64)
+        prev_out = (np.empty((cfg.B * cfg.Hkv, cfg.k), np.int32),
+                    np.empty((cfg.B * cfg.Hkv, cfg.k), np.int8), np.empty(cfg.B * cfg.Hkv))
         while True:
             qs = syn.query_step(cfg, t, prev, retry)
             q16 = syn.round_bf16(qs)
@@ -222,14 +234,16 @@ def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = M
                 rows = fc.reshape(cfg.B, cfg.Hkv, 1, cfg.d)
             else:
                 rows = q16.reshape(cfg.B, cfg.Hkv, G, cfg.d)
-            scores = orc.block_scores(rows)
-            _, _, gap = orc.select(scores, inp.evict[t], commit=False)
-            bad = (gap.reshape(cfg.B, cfg.Hkv) < margin) & pending
+            orc.block_scores(rows, out=scores, gmask=todo)
+            _, _, gap = orc.select(scores, inp.evict[t], commit=False, gmask=todo, out=prev_out)
+            bad = (gap < margin) & (todo != 0)
             if not bad.any():
                 break
-            if (retry[bad] >= max_retry).any():
+            bad2 = bad.reshape(cfg.B, cfg.Hkv)
+            if (retry[bad2] >= max_retry).any():
                 raise RuntimeError(f"{cfg.name}: no query with margin {margin} at step {t}")
-            retry[bad] += 1
+            retry[bad2] += 1
+            todo = bad.astype(np.uint8)
         prev = qs
         sel, src, gap = orc.select(scores, inp.evict[t], commit=True)
         miss = orc.residency(sel)

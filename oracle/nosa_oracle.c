@@ -151,7 +151,6 @@ int orc_init(const orc_cfg* c, orc_state* st, const int32_t* prefill_len, const 
       st->alive[(size_t)gi * nb + j] = 1;
       st->last_used[(size_t)gi * nb + j] = 0;
     }
-    for (int i = 0; i < MS; ++i) sub_mean(c, st, gi, i, st->kbar + ((size_t)gi * MS + i) * c->d);
     if (c->offload) {
       int used = 0;
       for (int z = 0; z < c->slots; ++z) st->slot_owner[(size_t)gi * c->slots + z] = -1;
@@ -167,6 +166,9 @@ int orc_init(const orc_cfg* c, orc_state* st, const int32_t* prefill_len, const 
       }
     }
   }
+#pragma omp parallel for schedule(dynamic) collapse(2)
+  for (int gi = 0; gi < NG; ++gi)
+    for (int i = 0; i < MS; ++i) sub_mean(c, st, gi, i, st->kbar + ((size_t)gi * MS + i) * c->d);
   return 0;
 }
 
@@ -183,12 +185,15 @@ void orc_append(const orc_cfg* c, orc_state* st, const uint16_t* k_new, const ui
   }
 }
 
-/* Block scores of the two-stage pool; blocks at or beyond N get -INFINITY. */
-void orc_block_scores(const orc_cfg* c, const orc_state* st, const uint16_t* rows, double* scores) {
+/* Block scores of the two-stage pool; blocks at or beyond N get -INFINITY.
+ * gmask (NULL = all) restricts the call to the groups with gmask[gi] != 0. */
+void orc_block_scores(const orc_cfg* c, const orc_state* st, const uint16_t* rows, double* scores,
+                      const uint8_t* gmask) {
   const int NG = n_groups(c), nb = c->max_blocks, MS = max_sub(c), spb = c->bs / c->s;
   const int R = c->n_rows;
 #pragma omp parallel for schedule(dynamic)
   for (int gi = 0; gi < NG; ++gi) {
+    if (gmask && !gmask[gi]) continue;
     const int L = st->len[gi];
     const int N = cdiv(L, c->bs), M = cdiv(L, c->s);
     double* out = scores + (size_t)gi * nb;
@@ -213,13 +218,14 @@ void orc_block_scores(const orc_cfg* c, const orc_state* st, const uint16_t* row
 /*
  * Dual selection. sel[gi][0..k) = S(t) ascending, padded with -1; src = 1 for
  * Gamma_e, 2 for Gamma_q, 0 for padding. gap_q = margin of the query-aware cut.
- * commit != 0 updates prev_sel and alive; commit == 0 only previews.
+ * commit != 0 updates prev_sel and alive; commit == 0 only previews. gmask as above.
  */
 void orc_select(const orc_cfg* c, orc_state* st, const double* scores, const float* evict,
-                int32_t* sel, int8_t* src, double* gap_q, int commit) {
+                int32_t* sel, int8_t* src, double* gap_q, int commit, const uint8_t* gmask) {
   const int NG = n_groups(c), nb = c->max_blocks, k = c->k_q + c->k_e;
 #pragma omp parallel for schedule(dynamic)
   for (int gi = 0; gi < NG; ++gi) {
+    if (gmask && !gmask[gi]) continue;
     const int L = st->len[gi];
     const int N = cdiv(L, c->bs);
     uint8_t* ps = st->prev_sel + (size_t)gi * nb;
