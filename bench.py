@@ -10,7 +10,8 @@ k_e=48, 8 planted high-affinity blocks per group), synthetic seeded inputs.
 
 Printed: one JSON line. `value` is queries/s (query-head vectors, B*Hq per
 step, summed over ranks) from CUDA-event time of the timed steps, inputs
-resident in HBM, L2 flushed (256 MiB write) before every timed step. `e2e` is
+resident in HBM, L2 flushed before every timed step (256 MiB written, then
+256 MiB read so the write-back of dirty lines happens before the timed region). `e2e` is
 the same metric with each step's inputs copied from pinned host memory and the
 outputs copied back inside the timed region. `roofline` is for the attention
 kernel (the largest share of the step), `cpu_baseline` times the fp64 oracle on
@@ -242,7 +243,19 @@ def run_gpu(args, cfg):
     sel = torch.empty(NG * cfg.k, dtype=torch.int32, device="cuda")
     out = torch.empty(cfg.B * cfg.Hq * cfg.d, dtype=torch.float32, device="cuda")
     miss = torch.empty(NG, dtype=torch.int32, device="cuda")
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    # L2 flush between timed steps: write a buffer larger than L2, then read another one so
+    # the dirty lines are written back before the timed region starts, not inside it
+    flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush_sink = torch.empty(1, dtype=torch.float32, device="cuda")
+
+    class _Flush:
+        @staticmethod
+        def zero_():
+            flush_w.zero_()
+            torch.sum(flush_r, dim=0, out=flush_sink)
+
+    flush = _Flush()
     stream = torch.cuda.current_stream()
 
     def do_step(t, events=None):
@@ -343,7 +356,7 @@ def run_gpu(args, cfg):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": describe(cfg), "global_batch": cfg.B * world, "seq_len": cfg.T[0],
                    "parallelism": f"replicas x{world} (batch-sharded, no collective)",
-                   "l2": "flushed (256 MiB write) before every timed step",
+                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read so no dirty line is written back inside the timed region)",
                    "queries_per_step": q_per_step},
         "step_us": 1e3 * tot_ms / args.steps,
         "step_us_median": 1e3 * float(np.median(step_ms)),

@@ -102,7 +102,7 @@ nosa_status check_state(const nosa_config& c, const nosa_state* st) {
 }
 
 struct WsLayout {
-  size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, total;
+  size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, ge_mask, total;
   int copy_stride;
 };
 
@@ -120,6 +120,7 @@ WsLayout ws_layout(const nosa_config& c) {
   w.copy_list = off; off += up256(NG * (size_t)w.copy_stride * 8);
   w.copy_count = off; off += up256(NG * 4);
   w.partials = off; off += up256(NG * kPartialSlots * (size_t)G * (c.d + 2) * 4);
+  w.ge_mask = off; off += up256(NG * (size_t)words(c) * 4);
   w.total = off;
   return w;
 }
@@ -171,6 +172,7 @@ void set_ws(StepArgs& a, const nosa_config& c, void* ws) {
   a.copy_stride = w.copy_stride;
   a.copy_count = ws_at<int32_t>(ws, w.copy_count);
   a.counters = ws_at<uint32_t>(ws, w.cnt_k1);
+  a.ge_mask = ws_at<uint32_t>(ws, w.ge_mask);
 }
 
 // ------------------------------------------------------------------ launches
@@ -204,14 +206,21 @@ nosa_status launch_sel_kernel(void (*k)(StepArgs), const nosa_config& c, const S
 nosa_status launch_copy(const nosa_config& c, const nosa_state* st, void* ws, cudaStream_t s) {
   const WsLayout w = ws_layout(c);
   const int page_vec = c.block_size * c.d * 2 / 16;
-  dim3 grid(n_groups(c), 8);
-  copy_kernel<<<grid, 256, 0, s>>>(ws_at<int2>(ws, w.copy_list), w.copy_stride,
-                                   ws_at<int32_t>(ws, w.copy_count),
-                                   reinterpret_cast<const uint4*>(st->host_k),
-                                   reinterpret_cast<const uint4*>(st->host_v),
-                                   reinterpret_cast<uint4*>(st->k_pool),
-                                   reinterpret_cast<uint4*>(st->v_pool), c.max_blocks, page_vec);
-  NOSA_CUDA(cudaGetLastError());
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(n_groups(c), 8);
+  lc.blockDim = dim3(256);
+  lc.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  NOSA_CUDA(cudaLaunchKernelEx(&lc, copy_kernel, (const int2*)ws_at<int2>(ws, w.copy_list), w.copy_stride,
+                               (const int32_t*)ws_at<int32_t>(ws, w.copy_count),
+                               reinterpret_cast<const uint4*>(st->host_k),
+                               reinterpret_cast<const uint4*>(st->host_v),
+                               reinterpret_cast<uint4*>(st->k_pool), reinterpret_cast<uint4*>(st->v_pool),
+                               c.max_blocks, page_vec));
   return NOSA_OK;
 }
 
@@ -259,6 +268,8 @@ nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& t
   const size_t smem = SH::smem_bytes(stages);
   auto k = attn_kernel<D, BS>;
   NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared));
   int dev = 0, sms = 0, per_sm = 0;
   NOSA_CUDA(cudaGetDevice(&dev));
   NOSA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
@@ -272,8 +283,17 @@ nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& t
   a.W = W;
   a.stages = stages;
   const int grid = (a.total + W - 1) / W;
-  k<<<grid, SH::THREADS, smem, s>>>(tk, tv, a);
-  NOSA_CUDA(cudaGetLastError());
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(SH::THREADS);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  NOSA_CUDA(cudaLaunchKernelEx(&lc, k, tk, tv, a));
   return NOSA_OK;
 }
 

@@ -13,10 +13,12 @@
 // Inside a CTA: one producer warp issues TMA tile loads (128-byte swizzle, no
 // multicast) of the K and V page of each task into a ring of shared-memory
 // stages; BS/16 consumer warps each own 16 tokens of every page. Per warp the
-// G query heads are the rows of an m16n8k16 bf16 mma (rows >= G are zero);
-// q.K^T uses K straight from shared memory (ldmatrix), P.V uses V through
-// ldmatrix.trans with P split into bf16 hi + lo parts so that P keeps ~16
-// mantissa bits (a single bf16 P would cost ~1e-3 relative error).
+// G query heads are rows 0..G-1 of an m16n8k16 bf16 mma (other rows zero);
+// q.K^T uses K straight from shared memory (ldmatrix). P.V uses V through
+// ldmatrix.trans with P split into bf16 hi + lo parts (a single bf16 P would
+// cost ~1e-3 relative error): rows 0..7 of the A operand carry P_hi and rows
+// 8..15 carry P_lo, so one mma accumulates both and the two halves of the
+// accumulator are summed when the partial is written.
 #pragma once
 
 #include "nosa_common.cuh"
@@ -71,7 +73,7 @@ __device__ __forceinline__ uint32_t swz(int row, int col) {
 }
 
 template <int D, int BS>
-__global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
+__global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
     attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 AttnArgs a) {
   using SH = AttnShape<D, BS>;
@@ -96,61 +98,82 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
     }
     fence_barrier_init();
   }
+  if (warp == NC && lane == 0) {
+    tma_prefetch_desc(&tmk);
+    tma_prefetch_desc(&tmv);
+  }
   __syncthreads();
+  griddep_wait();  // sel, seq_len and the block table come from the previous kernel
   const unsigned long long deadline = globaltimer() + kWaitLimitNs;
 
   if (warp == NC) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmk);
-      tma_prefetch_desc(&tmv);
-      int issued = 0;
-      for (int i = 0; i < ntask; ++i) {
-        const int s = i % ST, round = i / ST;
-        if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, deadline)) {
-          set_err(a.err, NOSA_ERR_TIMEOUT);
-          break;
-        }
-        const int t = task0 + i;
-        const int gi = t / a.k;
-        const int L = a.seq_len[gi];
-        const int N = (L + BS - 1) / BS;
-        int j = a.sel[t];
-        if (j >= N) {
+    // The warp resolves 32 tasks' metadata at once (sel -> block table, in parallel
+    // across lanes); lane 0 then issues the tile loads in task order.
+    int issued = 0;
+    bool abort = false;
+    for (int base = 0; base < ntask && !abort; base += 32) {
+      const int i_l = base + lane;
+      int gi_l = 0, j_l = -1, L_l = 0, page_l = -1;
+      if (i_l < ntask) {
+        const int t = task0 + i_l;
+        gi_l = t / a.k;
+        L_l = __ldg(a.seq_len + gi_l);
+        const int N = (L_l + BS - 1) / BS;
+        j_l = __ldg(a.sel + t);
+        if (j_l >= N) {
           set_err(a.err, NOSA_ERR_SEL);
-          j = -1;
+          j_l = -1;
         }
-        int page = -1;
-        if (j >= 0) {
-          page = a.block_table[(size_t)gi * a.max_blocks + j];
-          if (page < 0 || page >= a.total_pages) {
+        if (j_l >= 0) {
+          page_l = __ldg(a.block_table + (size_t)gi_l * a.max_blocks + j_l);
+          if (page_l < 0 || page_l >= a.total_pages) {
             set_err(a.err, NOSA_ERR_BLOCK_TABLE);
-            j = -1;
+            j_l = -1;
           }
         }
-        TaskInfo ti;
-        ti.gi = gi;
-        ti.j = j;
-        ti.L = L;
-        ti.last = (i == ntask - 1) || ((t + 1) / a.k != gi);
-        info[s] = ti;
-        if (j >= 0) {
-          mbar_arrive_expect_tx(&full[s], SH::STAGE);
-          uint8_t* st = smem + (size_t)s * SH::STAGE;
-#pragma unroll
-          for (int h = 0; h < SH::HALVES; ++h) {
-            tma_load_2d(st + h * SH::TILE, &tmk, &full[s], 64 * h, page * BS);
-            tma_load_2d(st + SH::KV + h * SH::TILE, &tmv, &full[s], 64 * h, page * BS);
-          }
-        } else {
-          mbar_arrive(&full[s]);
-        }
-        issued = i + 1;
       }
-      // never leave the CTA with a tile load in flight
+      const int nb = min(32, ntask - base);
+      for (int u = 0; u < nb; ++u) {
+        const int gi = __shfl_sync(0xffffffffu, gi_l, u);
+        const int j = __shfl_sync(0xffffffffu, j_l, u);
+        const int L = __shfl_sync(0xffffffffu, L_l, u);
+        const int page = __shfl_sync(0xffffffffu, page_l, u);
+        const int i = base + u;
+        if (lane == 0) {
+          const int s = i % ST, round = i / ST;
+          if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, deadline)) {
+            set_err(a.err, NOSA_ERR_TIMEOUT);
+            abort = true;
+          } else {
+            TaskInfo ti;
+            ti.gi = gi;
+            ti.j = j;
+            ti.L = L;
+            ti.last = (i == ntask - 1) || ((task0 + i + 1) / a.k != gi);
+            info[s] = ti;
+            if (j >= 0) {
+              mbar_arrive_expect_tx(&full[s], SH::STAGE);
+              uint8_t* st = smem + (size_t)s * SH::STAGE;
+#pragma unroll
+              for (int h = 0; h < SH::HALVES; ++h) {
+                tma_load_2d(st + h * SH::TILE, &tmk, &full[s], 64 * h, page * BS);
+                tma_load_2d(st + SH::KV + h * SH::TILE, &tmv, &full[s], 64 * h, page * BS);
+              }
+            } else {
+              mbar_arrive(&full[s]);
+            }
+            issued = i + 1;
+          }
+        }
+        abort = __shfl_sync(0xffffffffu, abort, 0);
+        if (abort) break;
+      }
+    }
+    // never leave the CTA with a tile load in flight
+    if (lane == 0)
       for (int i = max(0, issued - ST); i < issued; ++i)
         mbar_wait(&full[i % ST], (i / ST) & 1, deadline);
-    }
     return;
   }
 
@@ -208,8 +231,8 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
         for (int ks = 0; ks < KS; ++ks) {
           uint32_t b0, b1, b2, b3;
           ldsm_x4(kbase + swz<BS>(row, 16 * ks + 8 * (mi & 1)), b0, b1, b2, b3);
-          mma_16816(sc[0], qa[ks][0], qa[ks][1], b0, b1);
-          mma_16816(sc[1], qa[ks][0], qa[ks][1], b2, b3);
+          mma_16816(sc[0], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+          mma_16816(sc[1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
         }
       }
       // online softmax (log2 domain); row hrow, tokens 8*nt + 2*c4 + e
@@ -243,6 +266,8 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
       for (int n = 0; n < NT; ++n) {
         acc[n][0] *= alpha;
         acc[n][1] *= alpha;
+        acc[n][2] *= alpha;
+        acc[n][3] *= alpha;
       }
       // P as bf16 hi + lo (A operand rows = heads, k = 16 tokens)
       const uint32_t ah0 = pack_bf16(p[0][0], p[0][1]);
@@ -259,10 +284,8 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
         for (int np = 0; np < NT / 2; ++np) {
           uint32_t b0, b1, b2, b3;
           ldsm_x4_t(vbase + swz<BS>(row, 16 * np + 8 * (mi >> 1)), b0, b1, b2, b3);
-          mma_16816(acc[2 * np], ah0, ah2, b0, b1);
-          mma_16816(acc[2 * np], al0, al2, b0, b1);
-          mma_16816(acc[2 * np + 1], ah0, ah2, b2, b3);
-          mma_16816(acc[2 * np + 1], al0, al2, b2, b3);
+          mma_16816(acc[2 * np], ah0, al0, ah2, al2, b0, b1);
+          mma_16816(acc[2 * np + 1], ah0, al0, ah2, al2, b2, b3);
         }
       }
     }
@@ -282,8 +305,8 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
         }
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-          w[2 + 8 * n + 2 * c4] = acc[n][0];
-          w[3 + 8 * n + 2 * c4] = acc[n][1];
+          w[2 + 8 * n + 2 * c4] = acc[n][0] + acc[n][2];
+          w[3 + 8 * n + 2 * c4] = acc[n][1] + acc[n][3];
         }
       }
       wrote_smem = true;

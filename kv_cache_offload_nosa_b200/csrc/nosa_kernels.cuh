@@ -48,6 +48,7 @@ struct StepArgs {
   int32_t* copy_count;
   int32_t* miss_count;
   uint32_t* counters;
+  uint32_t* ge_mask;      // [B*Hkv][W] Gamma_e handed from chunk 0 to the last chunk
   uint32_t* err;
 };
 
@@ -68,6 +69,7 @@ __device__ void append_token(const StepArgs& a, int gi, int len0) {
     const uint16_t vx = a.v_new[(size_t)gi * D + x];
     float sum = 0.f;
     if (page >= 0 || a.host_k) {
+#pragma unroll 8
       for (int tau = t0; tau < pos; ++tau) {
         const int rr = tau - jb * a.bs;
         const uint16_t* src = (page >= 0) ? a.k_pool + ((size_t)page * a.bs + rr) * D
@@ -100,6 +102,26 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gi = blockIdx.y, c = blockIdx.x;
+  const int i0 = c * kChunkSub;
+  const int sub = lane / LPS, part = lane % LPS;
+  const float4* kcg = reinterpret_cast<const float4*>(a.kc + (size_t)gi * a.max_sub * D);
+
+  if (FUSED) griddep_launch_dependents();  // the next kernel may start its prologue
+  // first batch of kc loads goes out before anything that depends on seq_len
+  const int icap = min(i0 + kChunkSub, a.max_sub);
+  int base = i0 + warp * SPW;
+  float4 va[4], vb[4];
+  auto load_batch = [&](int bse, int lim, float4* xa, float4* xb) {
+    const int ia = bse + sub, ib = bse + PASS + sub;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int p4 = part + LPS * jj;
+      xa[jj] = (ia < lim) ? __ldcs(kcg + (size_t)ia * (D / 4) + p4) : make_float4(0, 0, 0, 0);
+      xb[jj] = (ib < lim) ? __ldcs(kcg + (size_t)ib * (D / 4) + p4) : make_float4(0, 0, 0, 0);
+    }
+  };
+  load_batch(base, icap, va, vb);
+
   const int len0 = a.seq_len[gi];
   int L = len0;
   if (FUSED) {
@@ -109,12 +131,19 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   const int M = (L + a.s - 1) / a.s;
   const int N = (L + a.bs - 1) / a.bs;
   const int spb = a.bs / a.s;
-  const int i0 = c * kChunkSub;
   const int i1 = min(i0 + kChunkSub, M);
+  const int Wmax = (a.max_blocks + 31) / 32;
 
+  if (FUSED && c == 0) {
+    // query-agnostic selection needs no block score: it overlaps the other chunks' streaming
+    const SelSmem S = sel_smem_carve(dsm, a.max_blocks);
+    select_evict(S, a.evict + (size_t)gi * a.max_blocks, a.prev_sel + (size_t)gi * Wmax,
+                 a.alive + (size_t)gi * Wmax, a.ge_mask + (size_t)gi * Wmax, N, a.k_e, Wmax);
+  }
   if (FUSED && L > len0 && (len0 / a.s) / kChunkSub == c) {
     append_token<D>(a, gi, len0);
     __syncthreads();
+    load_batch(base, icap, va, vb);  // the tail sub-block's mean just changed
   }
   for (int x = tid; x < D; x += kScoreThreads) {
     const uint16_t* r = a.rows + (size_t)gi * a.R * D + x;
@@ -125,7 +154,6 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   __syncthreads();
 
   if (i0 < i1) {
-    const int sub = lane / LPS, part = lane % LPS;
     float qr[16];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
@@ -133,16 +161,10 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) qr[4 * jj + e] = qbar[4 * p4 + e];
     }
-    const float4* kcg = reinterpret_cast<const float4*>(a.kc + (size_t)gi * a.max_sub * D);
-    for (int base = i0 + warp * SPW; base < i1; base += 2 * PASS) {
+    for (; base < i1; base += 2 * PASS) {
+      float4 na[4], nb[4];
+      load_batch(base + 2 * PASS, i1, na, nb);  // next batch in flight during this one
       const int ia = base + sub, ib = base + PASS + sub;
-      float4 va[4], vb[4];
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int p4 = part + LPS * jj;
-        va[jj] = (ia < i1) ? __ldcs(kcg + (size_t)ia * (D / 4) + p4) : make_float4(0, 0, 0, 0);
-        vb[jj] = (ib < i1) ? __ldcs(kcg + (size_t)ib * (D / 4) + p4) : make_float4(0, 0, 0, 0);
-      }
       float da = 0.f, db = 0.f;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
@@ -164,6 +186,11 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
         if (ia < i1) su[ia - i0] = da;
         if (ib < i1) su[ib - i0] = db;
       }
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        va[jj] = na[jj];
+        vb[jj] = nb[jj];
+      }
     }
   }
   __syncthreads();
@@ -181,7 +208,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   }
   if (!FUSED) return;
 
-  // last chunk of this group to finish runs the selection
+  // last chunk of this group to finish runs the query-aware selection
   __threadfence();
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(&a.counters[gi], 1u) == gridDim.x - 1);
@@ -189,11 +216,9 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   if (!s_last) return;
   __threadfence();
   const SelSmem S = sel_smem_carve(dsm, a.max_blocks);
-  const int Wmax = (a.max_blocks + 31) / 32;
   const int k = a.k_q + a.k_e;
-  select_group(S, a.block_scores + (size_t)gi * a.max_blocks, a.evict + (size_t)gi * a.max_blocks,
-               a.prev_sel + (size_t)gi * Wmax, a.alive + (size_t)gi * Wmax, a.sel + (size_t)gi * k,
-               N, a.k_e, k, Wmax);
+  select_query(S, a.block_scores + (size_t)gi * a.max_blocks, a.ge_mask + (size_t)gi * Wmax,
+               a.prev_sel + (size_t)gi * Wmax, a.sel + (size_t)gi * k, N, k, Wmax);
   if (a.host_k) {
     PlanArgs p;
     p.block_table = a.block_table + (size_t)gi * a.max_blocks;
@@ -239,9 +264,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(StepArgs a) {
   const SelSmem S = sel_smem_carve(dsm, a.max_blocks);
   const int Wmax = (a.max_blocks + 31) / 32;
   const int k = a.k_q + a.k_e;
-  select_group(S, a.block_scores + (size_t)gi * a.max_blocks, a.evict + (size_t)gi * a.max_blocks,
-               a.prev_sel + (size_t)gi * Wmax, a.alive + (size_t)gi * Wmax, a.sel + (size_t)gi * k,
-               N, a.k_e, k, Wmax);
+  select_evict(S, a.evict + (size_t)gi * a.max_blocks, a.prev_sel + (size_t)gi * Wmax,
+               a.alive + (size_t)gi * Wmax, nullptr, N, a.k_e, Wmax);
+  select_query(S, a.block_scores + (size_t)gi * a.max_blocks, nullptr, a.prev_sel + (size_t)gi * Wmax,
+               a.sel + (size_t)gi * k, N, k, Wmax);
 }
 
 __global__ void __launch_bounds__(kSelThreads) plan_kernel(StepArgs a) {
@@ -275,6 +301,8 @@ __global__ void __launch_bounds__(256) copy_kernel(const int2* copy_list, int co
                                                    const int32_t* copy_count, const uint4* host_k,
                                                    const uint4* host_v, uint4* k_pool, uint4* v_pool,
                                                    int max_blocks, int page_vec) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int gi = blockIdx.x;
   const int n = copy_count[gi];
   for (int i = blockIdx.y; i < n; i += gridDim.y) {

@@ -13,6 +13,7 @@
 namespace nosa {
 
 constexpr int kSelThreads = 256;
+constexpr int kSmallSel = 256;  // candidate sets up to this size use O(n^2) rank counting
 
 // Shared-memory scratch of the selection, carved from dynamic shared memory.
 struct SelSmem {
@@ -26,12 +27,14 @@ struct SelSmem {
   int* hist;         // [256]
   int* red;          // [33]
   int* sc;           // [8]
+  int* list;         // [kSmallSel] candidate indices (rank-count path)
+  uint32_t* lkey;    // [kSmallSel] their keys
 };
 
 __host__ __device__ inline size_t sel_smem_bytes(int max_blocks) {
   const size_t nbp = (size_t)((max_blocks + 31) / 32) * 32;
   const size_t W = nbp / 32;
-  return 4 * nbp + 6 * 4 * W + 4 * 256 + 4 * 33 + 4 * 8 + 16;
+  return 4 * nbp + 6 * 4 * W + 4 * 256 + 4 * 33 + 4 * 8 + 8 * kSmallSel + 16;
 }
 
 __device__ inline SelSmem sel_smem_carve(uint8_t* base, int max_blocks) {
@@ -49,6 +52,8 @@ __device__ inline SelSmem sel_smem_carve(uint8_t* base, int max_blocks) {
   s.hist = reinterpret_cast<int*>(p);
   s.red = s.hist + 256;
   s.sc = s.red + 33;
+  s.list = s.sc + 8;
+  s.lkey = reinterpret_cast<uint32_t*>(s.list + kSmallSel);
   return s;
 }
 
@@ -59,46 +64,49 @@ __device__ __forceinline__ uint32_t word_valid_mask(int w, int n) {
   return (1u << (n - lo)) - 1u;
 }
 
-// Top-m of key[] over the candidate bitmask cand[0..W): higher key first, equal keys to
-// the lower index. Writes the bitmask into out[0..W). Returns min(m, |cand|).
-// All threads of the CTA must call it; W <= blockDim.x.
-__device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, int W, int m) {
-  const int tid = threadIdx.x, nth = blockDim.x;
-  int cnt = 0;
-  for (int w = tid; w < W; w += nth) cnt += __popc(cand[w]);
-  const int total = block_sum(cnt, S.red);
-  if (m <= 0 || m >= total) {
-    for (int w = tid; w < W; w += nth) out[w] = (m <= 0) ? 0u : cand[w];
-    __syncthreads();
-    return m <= 0 ? 0 : total;
-  }
+// Exact top-m by radix select: the threshold key, 8 bits per pass with warp-aggregated
+// histogram updates, then the lowest-index keys equal to the threshold fill the remainder.
+// ORs the chosen bits into out[0..W) (out must be zeroed by the caller). Used when a
+// range bucket holds more than kSmallSel keys (e.g. many equal scores).
+__device__ void sel_topm_radix(const SelSmem& S, const uint32_t* cand, uint32_t* out, int W, int m) {
+  const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31;
   uint32_t prefix = 0, pmask = 0;
   int rem = m;
+  const int span = W * 32;
+  const int iters = (span + nth - 1) / nth;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += nth) S.hist[i] = 0;
     __syncthreads();
-    for (int j = tid; j < W * 32; j += nth) {
-      if ((cand[j >> 5] >> (j & 31)) & 1u) {
+    for (int it = 0; it < iters; ++it) {
+      const int j = it * nth + tid;
+      bool take = false;
+      uint32_t dig = 0;
+      if (j < span && ((cand[j >> 5] >> (j & 31)) & 1u)) {
         const uint32_t k = S.key[j];
-        if ((k & pmask) == prefix) atomicAdd(&S.hist[(k >> shift) & 255u], 1);
+        take = (k & pmask) == prefix;
+        dig = (k >> shift) & 255u;
+      }
+      const unsigned act = __ballot_sync(0xffffffffu, take);
+      if (take) {
+        const unsigned peers = __match_any_sync(act, dig);
+        if (lane == __ffs(peers) - 1) atomicAdd(&S.hist[dig], __popc(peers));
       }
     }
     __syncthreads();
     if (tid < 32) {
-      // lane owns bins 255-8*lane .. 248-8*lane (descending key order)
-      int c[8], s = 0;
+      int c[8], sum = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         c[i] = S.hist[255 - 8 * tid - i];
-        s += c[i];
+        sum += c[i];
       }
-      int incl = s;
+      int incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (tid >= o) incl += y;
       }
-      const int excl = incl - s;
+      const int excl = incl - sum;
       if (excl < rem && rem <= incl) {
         int acc = excl;
 #pragma unroll
@@ -118,7 +126,6 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
     rem = S.sc[1];
     __syncthreads();
   }
-  // keys above the threshold, plus the `rem` lowest-index keys equal to it
   uint32_t gt = 0, eq = 0;
   if (tid < W) {
     const uint32_t cw = cand[tid];
@@ -131,9 +138,9 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
     }
   }
   const int ne = __popc(eq);
-  const int before = block_exclusive_scan(ne, S.red, nullptr);
+  const int eb = block_exclusive_scan(ne, S.red, nullptr);
   if (tid < W) {
-    int take = rem - before;
+    int take = rem - eb;
     take = take < 0 ? 0 : (take > ne ? ne : take);
     uint32_t t = eq, keep = 0;
     for (int x = 0; x < take; ++x) {
@@ -141,15 +148,166 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
       keep |= low;
       t ^= low;
     }
-    out[tid] = gt | keep;
+    out[tid] |= gt | keep;
   }
   __syncthreads();
+}
+
+// Top-m of key[] over the candidate bitmask cand[0..W): higher key first, equal keys to
+// the lower index. Writes the bitmask into out[0..W). Returns min(m, |cand|).
+// All threads of the CTA must call it; W <= blockDim.x.
+//  1. one pass: candidate count, smallest and largest key;
+//  2. keys fall into 256 equal-width buckets spanning [min, max] (so scores of similar
+//     magnitude still spread out), a histogram finds the bucket holding the m-th key;
+//  3. buckets above it are taken whole; the boundary bucket's keys are ranked exactly
+//     against each other (or, if it holds more than kSmallSel keys, radix-selected).
+__device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, int W, int m) {
+  const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = nth >> 5;
+  const int span = W * 32;
+  // element-strided passes: the 32 lanes of a warp cover one bitmask word per iteration
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  int cnt = 0;
+  for (int j = tid; j < span; j += nth) {
+    if ((cand[j >> 5] >> (j & 31)) & 1u) {
+      const uint32_t k = S.key[j];
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+      ++cnt;
+    }
+  }
+  for (int i = tid; i < 256; i += nth) S.hist[i] = 0;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  }
+  uint32_t* ured = reinterpret_cast<uint32_t*>(S.red);
+  if (lane == 0) {
+    ured[warp] = kmin;
+    ured[8 + warp] = kmax;
+    S.red[16 + warp] = cnt;
+  }
+  if (tid == 0) S.sc[2] = 0;
+  __syncthreads();
+  int total = 0;
+  kmin = 0xffffffffu;
+  kmax = 0u;
+  for (int i = 0; i < nw; ++i) {
+    kmin = min(kmin, ured[i]);
+    kmax = max(kmax, ured[8 + i]);
+    total += S.red[16 + i];
+  }
+  if (m <= 0 || m >= total) {
+    for (int w = tid; w < W; w += nth) out[w] = (m <= 0) ? 0u : cand[w];
+    __syncthreads();
+    return m <= 0 ? 0 : total;
+  }
+  const uint32_t range = kmax - kmin;
+  const int shift = (range < 256u) ? 0 : (32 - __clz(range) - 8);
+  for (int j = tid; j < span; j += nth)
+    if ((cand[j >> 5] >> (j & 31)) & 1u) atomicAdd(&S.hist[(S.key[j] - kmin) >> shift], 1);
+  __syncthreads();
+  if (tid < 32) {
+    int c[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      c[i] = S.hist[255 - 8 * tid - i];
+      sum += c[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (tid >= o) incl += y;
+    }
+    const int excl = incl - sum;
+    if (excl < m && m <= incl) {
+      int acc = excl;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (acc + c[i] >= m) {
+          S.sc[0] = 255 - 8 * tid - i;  // boundary bucket
+          S.sc[1] = m - acc;            // keys still to take from it
+          S.sc[3] = c[i];               // its size
+          break;
+        }
+        acc += c[i];
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t bstar = static_cast<uint32_t>(S.sc[0]);
+  const int rem = S.sc[1], nb = S.sc[3];
+  const bool small = nb <= kSmallSel;
+  for (int base = 0; base < span; base += nth) {
+    const int j = base + tid;
+    bool take = false, bnd = false;
+    if (j < span && ((cand[j >> 5] >> (j & 31)) & 1u)) {
+      const uint32_t k = S.key[j];
+      const uint32_t bk = (k - kmin) >> shift;
+      take = bk > bstar;
+      bnd = bk == bstar;
+      if (bnd && small) {
+        const int slot = atomicAdd(&S.sc[2], 1);
+        S.list[slot] = j;
+        S.lkey[slot] = k;
+      }
+    }
+    const uint32_t tw = __ballot_sync(0xffffffffu, take);
+    const uint32_t bw = __ballot_sync(0xffffffffu, bnd);
+    if (lane == 0 && j < span) {
+      out[j >> 5] = tw;
+      if (!small) S.m2[j >> 5] = bw;
+    }
+  }
+  __syncthreads();
+  if (small) {
+    for (int t = tid; t < nb; t += nth) {
+      const uint32_t k = S.lkey[t];
+      const int j = S.list[t];
+      int rank = 0;
+      for (int u = 0; u < nb; ++u) {
+        const uint32_t o = S.lkey[u];
+        rank += (o > k) || (o == k && S.list[u] < j);
+      }
+      if (rank < rem) atomicOr(&out[j >> 5], 1u << (j & 31));
+    }
+    __syncthreads();
+  } else {
+    sel_topm_radix(S, S.m2, out, W, rem);
+  }
   return m;
 }
 
-// Writes the set bits of mask[0..W) in ascending order to dst[base + rank]; returns |mask|.
+// Writes the set bits of mask[0..W) in ascending order to dst[rank]; returns |mask|.
+// All threads must call it.
 __device__ int sel_compact(const SelSmem& S, const uint32_t* mask, int W, int32_t* dst) {
   const int tid = threadIdx.x;
+  if (W <= 32) {
+    // one warp, no block-wide scan
+    if (tid < 32) {
+      const uint32_t mw = (tid < W) ? mask[tid] : 0u;
+      const int c = __popc(mw);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      uint32_t t = mw;
+      int r = incl - c;
+      while (t) {
+        const int b = __ffs(t) - 1;
+        t &= t - 1;
+        dst[r++] = tid * 32 + b;
+      }
+      if (tid == 31) S.sc[4] = incl;
+    }
+    __syncthreads();
+    return S.sc[4];
+  }
   const uint32_t mw = (tid < W) ? mask[tid] : 0u;
   int total;
   const int before = block_exclusive_scan(__popc(mw), S.red, &total);
@@ -166,30 +324,52 @@ __device__ int sel_compact(const SelSmem& S, const uint32_t* mask, int W, int32_
   return total;
 }
 
-// Dual selection of one group. scores/evict: the group's rows (global). prev/alive: the
-// group's bitmask words (global, updated). sel: the group's k outputs. On return S.sset
-// holds S(t).
-__device__ void select_group(const SelSmem& S, const float* scores, const float* evict,
-                             uint32_t* prev, uint32_t* alive, int32_t* sel, int N, int k_e, int k,
-                             int Wmax) {
+// Query-agnostic half of the dual selection for one group: Gamma_e = top-k_e of the
+// eviction scores over C_e = S(t-1) & A(t-1); candidates left out leave A for good.
+// Writes Gamma_e to ge_out (global, [Wmax] words) and updates alive. Returns |Gamma_e|.
+__device__ int select_evict(const SelSmem& S, const float* evict, const uint32_t* prev, uint32_t* alive,
+                            uint32_t* ge_out, int N, int k_e, int Wmax) {
   const int tid = threadIdx.x, nth = blockDim.x;
   const int W = (N + 31) / 32;
+  for (int j = tid; j < N; j += nth) S.key[j] = ord_f32(__ldg(evict + j));
   for (int w = tid; w < Wmax; w += nth) {
     const uint32_t a = alive[w];
     S.m1[w] = a;
     S.cand[w] = prev[w] & a & word_valid_mask(w, N);
   }
-  for (int j = tid; j < N; j += nth) S.key[j] = ord_f32(__ldg(evict + j));
   __syncthreads();
   const int ne = sel_topm(S, S.cand, S.ge, W, k_e);
-  // candidates left out of Gamma_e leave the alive set for good
   for (int w = tid; w < Wmax; w += nth) {
     const uint32_t c = (w < W) ? S.cand[w] : 0u;
     const uint32_t g = (w < W) ? S.ge[w] : 0u;
     alive[w] = S.m1[w] & ~(c & ~g);
-    if (w < W) S.cand[w] = word_valid_mask(w, N) & ~g;
+    if (ge_out) ge_out[w] = g;
+  }
+  __syncthreads();
+  return ne;
+}
+
+// Query-aware half: Gamma_q = top-min(k - |Gamma_e|, N - |Gamma_e|) of the block scores over
+// [0, N) minus Gamma_e, S(t) = Gamma_e + Gamma_q written to prev and, ascending and padded
+// with -1, to sel. Gamma_e comes from ge (global words written earlier in the same launch by
+// another CTA) or, when ge is NULL, from S.ge. On return S.sset holds S(t).
+__device__ void select_query(const SelSmem& S, const float* scores, const uint32_t* ge, uint32_t* prev,
+                             int32_t* sel, int N, int k, int Wmax) {
+  const int tid = threadIdx.x, nth = blockDim.x;
+  const int W = (N + 31) / 32;
+  int ne = 0;
+  for (int w = tid; w < W; w += nth) {
+    const uint32_t g = ge ? __ldcg(ge + w) : S.ge[w];
+    S.ge[w] = g;
+    S.cand[w] = word_valid_mask(w, N) & ~g;
+    ne += __popc(g);
   }
   for (int j = tid; j < N; j += nth) S.key[j] = ord_f32(__ldcg(scores + j));
+  for (int o = 16; o >= 1; o >>= 1) ne += __shfl_xor_sync(0xffffffffu, ne, o);
+  if ((tid & 31) == 0) S.red[tid >> 5] = ne;
+  __syncthreads();
+  ne = 0;
+  for (int i = 0; i < (nth >> 5); ++i) ne += S.red[i];
   __syncthreads();
   const int mq = (k - ne < N - ne) ? k - ne : N - ne;
   sel_topm(S, S.cand, S.pick, W, mq);

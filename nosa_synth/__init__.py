@@ -209,7 +209,7 @@ def configs() -> dict:
                              cfg_id=51)
     c["ragged_offload"] = NosaConfig("ragged_offload", 3, 8, 2, 128, (1000, 4096, 37), 32, 16, 6,
                                      10, 6, slots=40, drift=0.05, cfg_id=52)
-    c["empty"] = NosaConfig("empty", 2, 4, 1, 64, (0, 5), 32, 16, 2, 2, 40, cfg_id=53)
+    c["empty"] = NosaConfig("empty", 2, 4, 1, 64, (0, 33), 32, 16, 2, 2, 70, cfg_id=53)
     c["bs128_d64"] = NosaConfig("bs128_d64", 2, 16, 2, 64, (3000, 2900), 128, 16, 3, 5, 4,
                                 recipe="sink", cfg_id=54)
     c["g8"] = NosaConfig("g8", 2, 16, 2, 128, (1500, 1537), 64, 32, 5, 6, 3, cfg_id=55)
