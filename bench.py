@@ -41,8 +41,10 @@ METRIC = "sparse decode attn: queries/s, step µs, achieved HBM GB/s (% of peak)
 L2_FLUSH_BYTES = 256 << 20
 
 
-def workload(name: str, steps: int) -> syn.NosaConfig:
+def workload(name: str, steps: int, batch: int = 0) -> syn.NosaConfig:
     base = syn.configs()[name]
+    if batch:  # smaller batch of the same layer (profiling captures)
+        base = base.with_(B=batch, T=base.T[:1] * batch)
     return base.with_(steps=steps)
 
 
@@ -194,14 +196,11 @@ def run_gpu(args, cfg):
     import torch.distributed as dist
     import kv_cache_offload_nosa_b200 as nosa
     from kv_cache_offload_nosa_b200 import build as nb
+    from kv_cache_offload_nosa_b200 import dist as D
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = D.rank_info()
     torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    D.init("nccl", timeout_s=300)
     nb.build()
     # each rank is an independent replica with its own seeded batch (weak scaling)
     if world > 1:
@@ -272,8 +271,7 @@ def run_gpu(args, cfg):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     Ls = []
-    if world > 1:
-        dist.barrier()
+    D.barrier()
     torch.cuda.synchronize()
     with Clocks(local) as clk:
         for i in range(args.steps):
@@ -284,8 +282,7 @@ def run_gpu(args, cfg):
             Ls.append(cfg.T[0] + t + 1)
             t += 1
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    D.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     tot_ms = sum(step_ms)
     # per-kernel times of the same step (instrumented steps, events between kernels)
@@ -331,10 +328,7 @@ def run_gpu(args, cfg):
         raise RuntimeError(f"device fault in timed steps: rc={rc} err={err}")
 
     # max over ranks
-    agg = torch.tensor([tot_ms, e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(agg, op=dist.ReduceOp.MAX)
-    tot_ms, e2e_ms = agg.tolist()
+    tot_ms, e2e_ms = D.max_over_ranks([tot_ms, e2e_ms], device="cuda")
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
@@ -387,6 +381,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="llama")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling only)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
@@ -394,7 +389,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    cfg = workload(args.workload, args.warmup + args.steps)
+    cfg = workload(args.workload, args.warmup + args.steps, args.batch)
     if args.impl == "reference":
         run_reference(args, cfg)
     else:
