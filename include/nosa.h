@@ -194,6 +194,25 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
                       const float* evict_scores, int32_t* sel, float* out, int32_t* miss_count,
                       void* workspace, size_t ws_bytes, void* stream, void* const* events);
 
+/*
+ * No-allocation variant of nosa_decode_attn (the pages have no counterpart: this is an
+ * integration aid). Some callers cannot call cudaMalloc when they run attention: code being
+ * captured into a CUDA graph, plugins inside a host framework that owns all device memory,
+ * or a latency-bound serving loop that must not allocate or synchronise. This entry point
+ * computes exactly what nosa_decode_attn computes but takes no workspace: its scratch (the
+ * split-K partials and the per-group counters) lives in a static device array of 8 MiB
+ * inside the library, which every GPU that loads the library keeps until the process exits.
+ * Limit: B*Hkv * (8 * G * (d + 2) * 4 bytes, rounded up to 256) plus B*Hkv * 4 bytes must fit
+ * in 8 MiB (about 500 groups at G = 4, d = 128); larger configurations get NOSA_ENOMEM and
+ * must use nosa_decode_attn with a workspace. Allocates nothing: no cudaMalloc, no cudaFree.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture. Every call
+ * shares the one array: it zeroes the counters it needs on `stream` before the kernel, and
+ * calls whose kernels overlap on the GPU (other streams, other threads) race on the scratch.
+ */
+nosa_status nosa_decode_attn_noalloc(const nosa_config* cfg, const nosa_state* st, const uint16_t* q,
+                                     const int32_t* sel, float* out, void* stream);
+
 /* Synchronises the stream, reads state->err into *err_out (may be NULL):
  * NOSA_OK, NOSA_EDEVICE or NOSA_ETIMEOUT. */
 nosa_status nosa_check_device(const nosa_state* st, void* stream, uint32_t* err_out);

@@ -24,7 +24,8 @@ ERR_BLOCK_TABLE, ERR_SEL, ERR_NO_VICTIM, ERR_TIMEOUT, ERR_FULL, ERR_INIT = 1, 2,
 
 EXPORTS = ("nosa_state_sizes", "nosa_workspace_size", "nosa_workspace_init", "nosa_state_init",
            "nosa_append", "nosa_score_blocks", "nosa_select", "nosa_gather", "nosa_decode_attn",
-           "nosa_step", "nosa_check_device", "nosa_status_string", "nosa_last_error")
+           "nosa_step", "nosa_check_device", "nosa_status_string", "nosa_last_error",
+           "nosa_decode_attn_noalloc")
 
 
 class nosa_config(ctypes.Structure):
@@ -77,6 +78,7 @@ def load(path: Optional[str] = None):
         "nosa_decode_attn": [cfgp, stp, vp, vp, vp, vp, sz, vp],
         "nosa_step": [cfgp, stp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp],
         "nosa_check_device": [stp, vp, ctypes.POINTER(ctypes.c_uint32)],
+        "nosa_decode_attn_noalloc": [cfgp, stp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -166,6 +168,16 @@ def gather(cfg, st, sel, miss_count, ws, ws_bytes, stream=None):
 def decode_attn(cfg, st, q, sel, out, ws, ws_bytes, stream=None):
     _check(load().nosa_decode_attn(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(sel),
                                    _ptr(out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def decode_attn_noalloc(cfg, st, q, sel, out, stream=None):
+    """nosa_decode_attn without a workspace (scratch in the library's static device array).
+
+    For callers that cannot allocate device memory when attention runs; see include/nosa.h
+    for the size limit and the rule that overlapping calls race on the shared scratch.
+    """
+    _check(load().nosa_decode_attn_noalloc(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(sel),
+                                           _ptr(out), _stream(stream)))
 
 
 def step(cfg, st, q, score_rows, k_new, v_new, evict, sel, out, miss_count, ws, ws_bytes,

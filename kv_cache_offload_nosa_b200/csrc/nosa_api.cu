@@ -559,3 +559,93 @@ nosa_status nosa_check_device(const nosa_state* st, void* stream, uint32_t* err_
 }
 
 }  // extern "C"
+
+// ====================================================================== no-allocation attention
+// nosa_decode_attn_noalloc: the split-K attention of nosa_decode_attn with its scratch (the
+// per-group online-softmax partials and the last-arriver counters) placed in the array below
+// instead of the caller's workspace. The array lives in this library's device image, so every
+// GPU that loads the library holds it until the process exits.
+#include <mutex>
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. In host code the array's name
+// is only a host-side stand-in, so the address is looked up once per device (with that device
+// current) and cached.
+nosa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  NOSA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(NOSA_EINVAL, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(NOSA_ECUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return NOSA_OK;
+}
+}  // namespace
+
+extern "C" nosa_status nosa_decode_attn_noalloc(const nosa_config* cfg, const nosa_state* st,
+                                                const uint16_t* q, const int32_t* sel, float* out,
+                                                void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  NOSA_CHECK(q && sel && out && aligned16(q) && aligned16(sel) && aligned16(out),
+             "q/sel/out NULL or misaligned");
+  const size_t NG = n_groups(c);
+  const size_t part_bytes = up256(NG * kPartialSlots * (size_t)(c.Hq / c.Hkv) * (c.d + 2) * 4);
+  const size_t need = part_bytes + up256(NG * 4);
+  if (need > kNoAllocScratchBytes)
+    return fail(NOSA_ENOMEM, "nosa_decode_attn_noalloc needs %zu bytes of static scratch; the limit is %zu "
+                "(use nosa_decode_attn with a workspace)", need, kNoAllocScratchBytes);
+  void* base = nullptr;
+  if ((r = noalloc_scratch(&base)) != NOSA_OK) return r;
+  cudaStream_t s = as_stream(stream);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(base) + part_bytes);
+  // the array keeps the previous call's contents: the last-arriver counters must start at zero
+  NOSA_CUDA(cudaMemsetAsync(counters, 0, NG * 4, s));
+  CUtensorMap tk, tv;
+  if ((r = make_pool_map(&tk, c, st->k_pool)) != NOSA_OK) return r;
+  if ((r = make_pool_map(&tv, c, st->v_pool)) != NOSA_OK) return r;
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = q;
+  a.sel = sel;
+  a.seq_len = st->seq_len;
+  a.block_table = st->block_table;
+  a.out = out;
+  a.partials = static_cast<float*>(base);
+  a.counters = counters;
+  a.err = st->err;
+  a.Hq = c.Hq;
+  a.Hkv = c.Hkv;
+  a.G = c.Hq / c.Hkv;
+  a.k = kk(c);
+  a.max_blocks = c.max_blocks;
+  a.total = n_groups(c) * kk(c);
+  a.total_pages = (long long)n_groups(c) * c.slots;
+  a.scale_log2 = c.scale * 1.4426950408889634f;
+  if (c.d == 128) {
+    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s);
+    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s);
+    return launch_attn_t<128, 128>(c, a, tk, tv, s);
+  }
+  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s);
+  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s);
+  return launch_attn_t<64, 128>(c, a, tk, tv, s);
+}
