@@ -102,7 +102,7 @@ nosa_status check_state(const nosa_config& c, const nosa_state* st) {
 }
 
 struct WsLayout {
-  size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, ge_mask, total;
+  size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, ge_mask, sel_flag, total;
   int copy_stride;
 };
 
@@ -121,6 +121,7 @@ WsLayout ws_layout(const nosa_config& c) {
   w.copy_count = off; off += up256(NG * 4);
   w.partials = off; off += up256(NG * kPartialSlots * (size_t)G * (c.d + 2) * 4);
   w.ge_mask = off; off += up256(NG * (size_t)words(c) * 4);
+  w.sel_flag = off; off += up256(NG * 4);
   w.total = off;
   return w;
 }
@@ -298,7 +299,7 @@ nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& t
 }
 
 nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16_t* q, const int32_t* sel,
-                        float* out, void* ws, cudaStream_t s) {
+                        float* out, void* ws, cudaStream_t s, bool flags = false) {
   CUtensorMap tk, tv;
   nosa_status r = make_pool_map(&tk, c, st->k_pool);
   if (r != NOSA_OK) return r;
@@ -323,6 +324,7 @@ nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16
   a.total = n_groups(c) * kk(c);
   a.total_pages = (long long)n_groups(c) * c.slots;
   a.scale_log2 = c.scale * 1.4426950408889634f;
+  a.sel_flag = flags ? ws_at<uint32_t>(ws, w.sel_flag) : nullptr;
   if (c.d == 128) {
     if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s);
     if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s);
@@ -539,11 +541,15 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   a.evict = evict;
   a.sel = sel;
   a.miss_count = miss_count;
+  // Without host pools the attention starts on each group as soon as that group's selection
+  // is published (per-group flags); with host pools it waits for the page copies.
+  const bool flags = !has_host(st) && !events;
+  a.sel_flag = flags ? ws_at<uint32_t>(ws, ws_layout(c).sel_flag) : nullptr;
   if ((r = launch_score<true>(c, a, s)) != NOSA_OK) return r;
   if ((r = rec(1)) != NOSA_OK) return r;
   if (has_host(st) && (r = launch_copy(c, st, ws, s)) != NOSA_OK) return r;
   if ((r = rec(2)) != NOSA_OK) return r;
-  if ((r = launch_attn(c, st, q, sel, out, ws, s)) != NOSA_OK) return r;
+  if ((r = launch_attn(c, st, q, sel, out, ws, s, flags)) != NOSA_OK) return r;
   return rec(3);
 }
 

@@ -42,6 +42,7 @@ struct AttnArgs {
   int stages;
   long long total_pages;
   float scale_log2;           // sigma * log2(e)
+  uint32_t* sel_flag;         // [B*Hkv] per-group "selection published" flags, or NULL
 };
 
 struct TaskInfo {
@@ -103,7 +104,10 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
     tma_prefetch_desc(&tmv);
   }
   __syncthreads();
-  griddep_wait();  // sel, seq_len and the block table come from the previous kernel
+  // sel, seq_len, the block table and the appended token come from the previous kernel:
+  // either wait for that whole grid, or (flags) for the one group a task belongs to
+  const bool flags = a.sel_flag != nullptr;
+  if (!flags) griddep_wait();
   const unsigned long long deadline = globaltimer() + kWaitLimitNs;
 
   if (warp == NC) {
@@ -118,15 +122,16 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
       if (i_l < ntask) {
         const int t = task0 + i_l;
         gi_l = t / a.k;
-        L_l = __ldg(a.seq_len + gi_l);
+        if (flags && !wait_flag(a.sel_flag + gi_l, deadline)) set_err(a.err, NOSA_ERR_TIMEOUT);
+        L_l = __ldcg(a.seq_len + gi_l);
         const int N = (L_l + BS - 1) / BS;
-        j_l = __ldg(a.sel + t);
+        j_l = __ldcg(a.sel + t);
         if (j_l >= N) {
           set_err(a.err, NOSA_ERR_SEL);
           j_l = -1;
         }
         if (j_l >= 0) {
-          page_l = __ldg(a.block_table + (size_t)gi_l * a.max_blocks + j_l);
+          page_l = __ldcg(a.block_table + (size_t)gi_l * a.max_blocks + j_l);
           if (page_l < 0 || page_l >= a.total_pages) {
             set_err(a.err, NOSA_ERR_BLOCK_TABLE);
             j_l = -1;
@@ -134,6 +139,8 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
         }
       }
       const int nb = min(32, ntask - base);
+      __syncwarp();
+      if (flags && lane == 0) fence_proxy_async_global();  // pages written before the flags
       for (int u = 0; u < nb; ++u) {
         const int gi = __shfl_sync(0xffffffffu, gi_l, u);
         const int j = __shfl_sync(0xffffffffu, j_l, u);
@@ -357,7 +364,10 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
             }
           a.out[((size_t)b * a.Hq + g * a.G + h) * D + col] = (den > 0.f) ? num / den : 0.f;
         }
-        if (tid == 0) a.counters[gi] = 0u;
+        if (tid == 0) {
+          a.counters[gi] = 0u;
+          if (flags) a.sel_flag[gi] = 0u;  // every CTA of this group has passed its wait
+        }
       }
       named_bar(1, NC * 32);
     }

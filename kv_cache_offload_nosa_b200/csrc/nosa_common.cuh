@@ -88,6 +88,27 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Orders this thread's view of global memory (acquired from another CTA) before its later
+// async-proxy (TMA) reads of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Bounded wait for *flag != 0 (acquire). False once the deadline has passed.
+__device__ __forceinline__ bool wait_flag(const uint32_t* flag, unsigned long long deadline) {
+  for (uint32_t i = 0;; ++i) {
+    if (ld_acquire_gpu(flag) != 0u) return true;
+    if ((i & 15u) == 15u && globaltimer() > deadline) return false;
+    __nanosleep(64);
+  }
+}
 
 // ------------------------------------------------------------------ mma.sync fragments
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,

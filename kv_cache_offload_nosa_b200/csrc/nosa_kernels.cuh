@@ -49,6 +49,7 @@ struct StepArgs {
   int32_t* miss_count;
   uint32_t* counters;
   uint32_t* ge_mask;      // [B*Hkv][W] Gamma_e handed from chunk 0 to the last chunk
+  uint32_t* sel_flag;     // [B*Hkv] set (release) once a group's selection is published, or NULL
   uint32_t* err;
 };
 
@@ -240,6 +241,14 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   if (tid == 0) {
     a.counters[gi] = 0u;
     a.seq_len[gi] = L;
+  }
+  if (a.sel_flag) {
+    // everything the attention reads for this group is written: publish it
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      st_release_gpu(a.sel_flag + gi, 1u);
+    }
   }
 }
 

@@ -177,12 +177,10 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
     }
   }
   for (int i = tid; i < 256; i += nth) S.hist[i] = 0;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  }
+  // single-instruction warp reductions (redux.sync) instead of shuffle trees
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  cnt = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
   uint32_t* ured = reinterpret_cast<uint32_t*>(S.red);
   if (lane == 0) {
     ured[warp] = kmin;
@@ -268,6 +266,7 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
       const uint32_t k = S.lkey[t];
       const int j = S.list[t];
       int rank = 0;
+#pragma unroll 8
       for (int u = 0; u < nb; ++u) {
         const uint32_t o = S.lkey[u];
         rank += (o > k) || (o == k && S.list[u] < j);
@@ -331,6 +330,7 @@ __device__ int select_evict(const SelSmem& S, const float* evict, const uint32_t
                             uint32_t* ge_out, int N, int k_e, int Wmax) {
   const int tid = threadIdx.x, nth = blockDim.x;
   const int W = (N + 31) / 32;
+#pragma unroll 4
   for (int j = tid; j < N; j += nth) S.key[j] = ord_f32(__ldg(evict + j));
   for (int w = tid; w < Wmax; w += nth) {
     const uint32_t a = alive[w];
@@ -364,6 +364,7 @@ __device__ void select_query(const SelSmem& S, const float* scores, const uint32
     S.cand[w] = word_valid_mask(w, N) & ~g;
     ne += __popc(g);
   }
+#pragma unroll 4
   for (int j = tid; j < N; j += nth) S.key[j] = ord_f32(__ldcg(scores + j));
   for (int o = 16; o >= 1; o >>= 1) ne += __shfl_xor_sync(0xffffffffu, ne, o);
   if ((tid & 31) == 0) S.red[tid >> 5] = ne;
