@@ -277,8 +277,22 @@ nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& t
   NOSA_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, SH::THREADS, smem));
   if (per_sm < 1) per_sm = 1;
   const long long target = (long long)sms * per_sm;
-  int W = c.attn_split > 0 ? c.attn_split : (int)((a.total + target - 1) / target);
   const int wmin = (a.k + kPartialSlots - 2) / (kPartialSlots - 1);
+  int W = c.attn_split;
+  if (W <= 0) {
+    // Prefer a divisor of k: every CTA then holds one segment of one group and never flushes
+    // in mid-stream. Aim at about two CTAs per resident slot (finer work overlaps the
+    // selection tails of the score kernel and balances the end of the grid).
+    const double want = (double)a.total / (2.0 * (double)target);
+    int best = 0;
+    double best_d = 1e30;
+    for (int d = wmin; d <= a.k; ++d) {
+      if (a.k % d) continue;
+      const double dist = d > want ? d / want : want / d;
+      if (dist < best_d) { best_d = dist; best = d; }
+    }
+    W = (best > 0 && best_d <= 2.0) ? best : (int)((a.total + target - 1) / target);
+  }
   if (W < wmin) W = wmin;
   if (W < 1) W = 1;
   a.W = W;
