@@ -124,6 +124,27 @@ class Clocks:
                 "reasons": sorted(reasons)}
 
 
+def attn_traffic(batch: int):
+    """DRAM bytes per attention launch from the committed ncu summary, scaled from its batch to
+    `batch` (traffic grows with the number of groups); None when the kernel source changed
+    since the capture."""
+    import hashlib
+    import re
+    p = os.path.join(ROOT, "profiles", "attn_kernel_llama_b8.md")
+    if not os.path.exists(p):
+        return None
+    m = re.search(r"traffic-record: batch=(\d+) dram_bytes_per_launch=(\d+) source_sha256=([0-9a-f]+)",
+                  open(p).read())
+    if not m:
+        return None
+    h = hashlib.sha256()
+    for f in ("nosa_attn.cuh", "nosa_common.cuh"):
+        h.update(open(os.path.join(ROOT, "kv_cache_offload_nosa_b200", "csrc", f), "rb").read())
+    if h.hexdigest() != m.group(3):
+        return None
+    return int(m.group(2)) * batch / int(m.group(1))
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -359,7 +380,8 @@ def run_gpu(args, cfg):
         "kernel_us": {"score_select": 1e3 * float(np.mean(k_score)),
                       "gather": 1e3 * float(np.mean(k_gather)), "attention": 1e3 * attn_ms},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "attn_kernel",
+                     "frac": achieved / hbm_peak, "traffic": attn_traffic(cfg.B) if cfg.name == "llama" else None,
+                     "kernel": "attn_kernel",
                      "peak_kind": peak_kind,
                      "bytes_per_launch": float(np.mean(attn_b))},
         "e2e": {"value": q_per_step / (e2e_ms / 1e3), "unit": "queries/s",

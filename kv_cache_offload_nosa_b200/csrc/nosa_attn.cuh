@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
       m_run = -INFINITY;
       l_run = 0.f;
     }
-    bool wrote_smem = false;
+    bool wrote_smem = false, released = false;
     const int tok0 = ti.j * BS + 16 * warp;
     const int nval = (ti.j >= 0) ? min(16, ti.L - tok0) : 0;
     if (nval > 0) {
@@ -258,23 +258,28 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float m_new = fmaxf(m_run, mx);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = exp2f(m_run - m_use);
+      const float alpha = (m_new != m_run) ? ex2(m_run - m_use) : 1.f;
       float psum = 0.f;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          p[nt][e] = exp2f(p[nt][e] - m_use);
+          p[nt][e] = ex2(p[nt][e] - m_use);
           psum += p[nt][e];
         }
       l_run = l_run * alpha + psum;
+      // the running max of most rows stops moving after the first blocks: rescale only when
+      // some row's max changed (alpha == 1 exactly otherwise)
+      const bool moved = m_new != m_run;
       m_run = m_new;
+      if (__any_sync(0xffffffffu, moved)) {
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        acc[n][0] *= alpha;
-        acc[n][1] *= alpha;
-        acc[n][2] *= alpha;
-        acc[n][3] *= alpha;
+        for (int n = 0; n < NT; ++n) {
+          acc[n][0] *= alpha;
+          acc[n][1] *= alpha;
+          acc[n][2] *= alpha;
+          acc[n][3] *= alpha;
+        }
       }
       // P as bf16 hi + lo (A operand rows = heads, k = 16 tokens)
       const uint32_t ah0 = pack_bf16(p[0][0], p[0][1]);
@@ -342,6 +347,13 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
         }
         part[e] = v;
       }
+      // the scratch in stage s has been read by everyone: hand the stage back to the producer
+      // now, so the ticket and the combine below overlap the next tiles' loads
+      named_bar(1, NC * 32);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      released = true;
       __threadfence();
       named_bar(1, NC * 32);
       if (tid == 0) *s_flag = (atomicAdd(&a.counters[gi], 1u) == (unsigned)(nseg - 1));
@@ -371,9 +383,11 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
       }
       named_bar(1, NC * 32);
     }
-    if (wrote_smem) fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    if (!released) {
+      if (wrote_smem) fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
   }
 }
 
