@@ -153,15 +153,47 @@ __device__ void sel_topm_radix(const SelSmem& S, const uint32_t* cand, uint32_t*
   __syncthreads();
 }
 
+// Inverse of ord_f32 for keys of finite floats.
+__device__ __forceinline__ float key_f32(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Bucket of a key among 256 over [kmin, kmax]. Any map that never decreases as the key grows
+// keeps the selection exact: keys in a higher bucket are strictly larger than keys in a lower
+// one, and the boundary bucket is ranked exactly. Float keys (scores) use equal-width buckets
+// in value, so a bell-shaped set of scores spreads over many buckets and the boundary bucket
+// holds a handful of keys; other keys use the top 8 bits of (key - kmin).
+struct KeyBuckets {
+  uint32_t kmin;
+  int shift;
+  float vlo, inv;
+  bool lin;
+  __device__ KeyBuckets(uint32_t lo, uint32_t hi, bool float_keys) : kmin(lo) {
+    const uint32_t range = hi - lo;
+    shift = (range < 256u) ? 0 : (32 - __clz(range) - 8);
+    vlo = key_f32(lo);
+    const float vhi = key_f32(hi), span = vhi - vlo;
+    inv = 256.0f / span;
+    lin = float_keys && isfinite(vlo) && isfinite(vhi) && span > 0.0f && isfinite(span) &&
+          isfinite(inv) && inv > 0.0f;
+  }
+  __device__ __forceinline__ uint32_t operator()(uint32_t k) const {
+    if (lin) return min(255u, static_cast<uint32_t>(__float2int_rz((key_f32(k) - vlo) * inv)));
+    return (k - kmin) >> shift;
+  }
+};
+
 // Top-m of key[] over the candidate bitmask cand[0..W): higher key first, equal keys to
 // the lower index. Writes the bitmask into out[0..W). Returns min(m, |cand|).
-// All threads of the CTA must call it; W <= blockDim.x.
+// All threads of the CTA must call it; W <= blockDim.x. float_keys: the keys are ord_f32
+// images of floats.
 //  1. one pass: candidate count, smallest and largest key;
-//  2. keys fall into 256 equal-width buckets spanning [min, max] (so scores of similar
-//     magnitude still spread out), a histogram finds the bucket holding the m-th key;
+//  2. keys fall into 256 buckets spanning [min, max] (KeyBuckets), a histogram finds the
+//     bucket holding the m-th key;
 //  3. buckets above it are taken whole; the boundary bucket's keys are ranked exactly
 //     against each other (or, if it holds more than kSmallSel keys, radix-selected).
-__device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, int W, int m) {
+__device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, int W, int m,
+                        bool float_keys) {
   const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int nw = nth >> 5;
   const int span = W * 32;
@@ -202,10 +234,9 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
     __syncthreads();
     return m <= 0 ? 0 : total;
   }
-  const uint32_t range = kmax - kmin;
-  const int shift = (range < 256u) ? 0 : (32 - __clz(range) - 8);
+  const KeyBuckets bucket(kmin, kmax, float_keys);
   for (int j = tid; j < span; j += nth)
-    if ((cand[j >> 5] >> (j & 31)) & 1u) atomicAdd(&S.hist[(S.key[j] - kmin) >> shift], 1);
+    if ((cand[j >> 5] >> (j & 31)) & 1u) atomicAdd(&S.hist[bucket(S.key[j])], 1);
   __syncthreads();
   if (tid < 32) {
     int c[8], sum = 0;
@@ -244,7 +275,7 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
     bool take = false, bnd = false;
     if (j < span && ((cand[j >> 5] >> (j & 31)) & 1u)) {
       const uint32_t k = S.key[j];
-      const uint32_t bk = (k - kmin) >> shift;
+      const uint32_t bk = bucket(k);
       take = bk > bstar;
       bnd = bk == bstar;
       if (bnd && small) {
@@ -338,7 +369,7 @@ __device__ int select_evict(const SelSmem& S, const float* evict, const uint32_t
     S.cand[w] = prev[w] & a & word_valid_mask(w, N);
   }
   __syncthreads();
-  const int ne = sel_topm(S, S.cand, S.ge, W, k_e);
+  const int ne = sel_topm(S, S.cand, S.ge, W, k_e, true);
   for (int w = tid; w < Wmax; w += nth) {
     const uint32_t c = (w < W) ? S.cand[w] : 0u;
     const uint32_t g = (w < W) ? S.ge[w] : 0u;
@@ -373,7 +404,7 @@ __device__ void select_query(const SelSmem& S, const float* scores, const uint32
   for (int i = 0; i < (nth >> 5); ++i) ne += S.red[i];
   __syncthreads();
   const int mq = (k - ne < N - ne) ? k - ne : N - ne;
-  sel_topm(S, S.cand, S.pick, W, mq);
+  sel_topm(S, S.cand, S.pick, W, mq, true);
   for (int w = tid; w < Wmax; w += nth) {
     const uint32_t s = (w < W) ? (S.ge[w] | S.pick[w]) : 0u;
     S.sset[w] = s;
@@ -463,7 +494,7 @@ __device__ void plan_group(const SelSmem& S, const PlanArgs& p) {
         if ((v >> b) & 1u) S.key[w * 32 + b] = ord_lru(p.last_used[w * 32 + b]);
     }
     __syncthreads();
-    const int got = sel_topm(S, S.m2, S.ge, W, nv);
+    const int got = sel_topm(S, S.m2, S.ge, W, nv, false);
     if (got < nv) {
       set_err(p.err, NOSA_ERR_NO_VICTIM);
       nv = got;
