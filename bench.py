@@ -54,10 +54,12 @@ def describe(cfg: syn.NosaConfig) -> str:
             + (f" slots={cfg.slots} offload" if cfg.offload else " all KV in HBM"))
 
 
-def step_bytes(cfg: syn.NosaConfig, L: int):
+def step_bytes(cfg: syn.NosaConfig, L: int, misses: int = 0):
     """Algorithmic bytes of one step at context length L (after the append), per step.
 
-    Returns (total, attention kernel, score/select kernel)."""
+    `misses`: pages (K and V each) the step copied from host memory; each is read over PCIe
+    once and written to HBM once. Returns (total HBM, attention kernel, score/select kernel,
+    PCIe)."""
     NG, G, d, bs = cfg.B * cfg.Hkv, cfg.G, cfg.d, cfg.block
     N = -(-L // bs)
     M = -(-L // cfg.sub_block)
@@ -69,7 +71,26 @@ def step_bytes(cfg: syn.NosaConfig, L: int):
     attn = NG * (kv + G * d * 2 + G * d * 4 + cfg.k * 4 + cfg.k * 4)
     score = NG * (M * d * 4 + N * 4 + 2 * 2 * 4 * (-(-N // 32)) + cfg.rows * d * 2
                   + 2 * d * 2 + N * 4 * 2 + cfg.k * 4)
-    return attn + score, attn, score
+    page = bs * d * 2
+    return attn + score + misses * 2 * page, attn, score, misses * 2 * page
+
+
+def pcie_ceiling(nosa, torch, mib: int = 256, reps: int = 5):
+    """PCIe read ceiling: best rate of the library's plain UVA read probe (16-byte loads from
+    pinned host memory, the gather's access) over `mib` MiB, CUDA events."""
+    n = mib << 20
+    h = torch.empty(n, dtype=torch.uint8).pin_memory()
+    dv = torch.empty(n, dtype=torch.uint8, device="cuda")
+    rates = []
+    for i in range(reps + 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        nosa.uva_read_probe(h, dv, n)
+        b.record()
+        torch.cuda.synchronize()
+        if i:
+            rates.append(n / (a.elapsed_time(b) / 1e3) / 1e9)
+    return max(rates)
 
 
 class Clocks:
@@ -249,6 +270,28 @@ def run_gpu(args, cfg):
     inp.pool_k = inp.pool_v = None
     plen = torch.tensor(cfg.T, dtype=torch.int32, device="cuda")
     cache.init(plen, resident)
+    if cfg.offload:
+        # the first launch of each kernel loads its module: do that on a small cache of the same
+        # shapes so that step 0 below is timed without it
+        small = syn.configs()["offload_small"].with_(steps=2)
+        si = syn.make_inputs(small)
+        sc = nosa.make_config(small.B, small.Hq, small.Hkv, small.d, small.block, small.sub_block,
+                              small.k_q, small.k_e, small.max_blocks, slots=small.n_slots,
+                              n_score_rows=small.rows, scale=small.scale)
+        scache = nosa.NosaCache(sc, offload=True)
+        sng = small.B * small.Hkv
+        scache.pool_view("host_k").copy_(torch.from_numpy(si.pool_k.reshape(sng, small.max_blocks, small.block, small.d)).view(torch.int16))
+        scache.pool_view("host_v").copy_(torch.from_numpy(si.pool_v.reshape(sng, small.max_blocks, small.block, small.d)).view(torch.int16))
+        scache.init(torch.tensor(small.T, dtype=torch.int32, device="cuda"),
+                    torch.from_numpy(si.resident.reshape(sng, -1)).cuda())
+        sq = torch.from_numpy(syn.round_bf16(syn.query_step(small, 0, None, np.zeros((small.B, small.Hkv), np.int64)))).view(torch.int16).cuda()
+        scache.step(sq, torch.from_numpy(si.k_new[0]).view(torch.int16).cuda(),
+                    torch.from_numpy(si.v_new[0]).view(torch.int16).cuda(), torch.from_numpy(si.evict[0]).cuda(),
+                    torch.empty(sng * small.k, dtype=torch.int32, device="cuda"),
+                    torch.empty(small.B * small.Hq * small.d, dtype=torch.float32, device="cuda"),
+                    torch.empty(sng, dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+        del scache
     # per-step inputs (queries follow the workload's process, no margin redraws)
     prev, zero = None, np.zeros((cfg.B, cfg.Hkv), np.int64)
     qs = []
@@ -262,7 +305,9 @@ def run_gpu(args, cfg):
     d_q, d_kn, d_vn, d_ev = (x.cuda() for x in (h_q, h_kn, h_vn, h_ev))
     sel = torch.empty(NG * cfg.k, dtype=torch.int32, device="cuda")
     out = torch.empty(cfg.B * cfg.Hq * cfg.d, dtype=torch.float32, device="cuda")
-    miss = torch.empty(NG, dtype=torch.int32, device="cuda")
+    # every step writes its miss counts to its own row (nothing extra runs in the timed region)
+    # (rows padded to 16 bytes: the library wants 16-byte aligned buffers)
+    miss_all = torch.zeros((total_steps, -(-NG // 4) * 4), dtype=torch.int32, device="cuda")
     # L2 flush between timed steps: write a buffer larger than L2, then read another one so
     # the dirty lines are written back before the timed region starts, not inside it
     flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -279,12 +324,22 @@ def run_gpu(args, cfg):
     stream = torch.cuda.current_stream()
 
     def do_step(t, events=None):
-        cache.step(d_q[t], d_kn[t], d_vn[t], d_ev[t], sel, out, miss, stream=stream, events=events)
+        cache.step(d_q[t], d_kn[t], d_vn[t], d_ev[t], sel, out, miss_all[t, :NG], stream=stream, events=events)
 
     t = 0
-    for _ in range(args.warmup):
+    # step 0 (S(-1) = every prefill block; with offload, the initial residency misses) is the
+    # first warm-up step, timed on its own
+    s0, e0_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush.zero_()
+    s0.record(stream)
+    do_step(t)
+    e0_.record(stream)
+    t += 1
+    for _ in range(args.warmup - 1):
         do_step(t)
         t += 1
+    torch.cuda.synchronize()
+    step0_ms = s0.elapsed_time(e0_)
     torch.cuda.synchronize()
     rc, err = cache.check()
     if rc != 0:
@@ -300,7 +355,7 @@ def run_gpu(args, cfg):
             starts[i].record(stream)
             do_step(t)
             ends[i].record(stream)
-            Ls.append(cfg.T[0] + t + 1)
+            Ls.append((cfg.T[0] + t + 1, t))
             t += 1
         torch.cuda.synchronize()
     D.barrier()
@@ -316,7 +371,7 @@ def run_gpu(args, cfg):
     for i in range(n_prof):
         flush.zero_()
         do_step(t, events=evs[i])
-        prof_L.append(cfg.T[0] + t + 1)
+        prof_L.append((cfg.T[0] + t + 1, t))
         t += 1
     torch.cuda.synchronize()
     k_score = [e[0].elapsed_time(e[1]) for e in evs]
@@ -326,7 +381,7 @@ def run_gpu(args, cfg):
     hp = [x.pin_memory() for x in (h_q, h_kn, h_vn, h_ev)]
     o_host = torch.empty(out.numel(), dtype=torch.float32, pin_memory=True)
     s_host = torch.empty(sel.numel(), dtype=torch.int32, pin_memory=True)
-    m_host = torch.empty(miss.numel(), dtype=torch.int32, pin_memory=True)
+    m_host = torch.empty(NG, dtype=torch.int32, pin_memory=True)
     bq, bk, bv, be = (torch.empty_like(x[0], device="cuda") for x in hp)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -336,10 +391,10 @@ def run_gpu(args, cfg):
         bk.copy_(hp[1][t], non_blocking=True)
         bv.copy_(hp[2][t], non_blocking=True)
         be.copy_(hp[3][t], non_blocking=True)
-        cache.step(bq, bk, bv, be, sel, out, miss, stream=stream)
+        cache.step(bq, bk, bv, be, sel, out, miss_all[t, :NG], stream=stream)
         o_host.copy_(out, non_blocking=True)
         s_host.copy_(sel, non_blocking=True)
-        m_host.copy_(miss, non_blocking=True)
+        m_host.copy_(miss_all[t, :NG], non_blocking=True)
         t += 1
     e1.record(stream)
     torch.cuda.synchronize()
@@ -348,6 +403,8 @@ def run_gpu(args, cfg):
     if rc != 0:
         raise RuntimeError(f"device fault in timed steps: rc={rc} err={err}")
 
+    misses = miss_all.sum(dim=1).cpu().numpy()  # K (and V) pages copied per step
+    pcie_peak = pcie_ceiling(nosa, torch) if cfg.offload else None
     # max over ranks
     tot_ms, e2e_ms = D.max_over_ranks([tot_ms, e2e_ms], device="cuda")
     if rank != 0:
@@ -357,11 +414,33 @@ def run_gpu(args, cfg):
     q_per_step = cfg.B * cfg.Hq * world
     value = q_per_step * args.steps / (tot_ms / 1e3)
     hbm_peak, peak_kind = peaks()
-    step_b = [step_bytes(cfg, L)[0] for L in Ls]
+    step_b = [step_bytes(cfg, L, int(misses[ti]))[0] for L, ti in Ls]
+    pcie_b = [step_bytes(cfg, L, int(misses[ti]))[3] for L, ti in Ls]
     hbm_gbs = sum(step_b) / (tot_ms / 1e3) / 1e9
-    attn_b = [step_bytes(cfg, L)[1] for L in prof_L]
+    attn_b = [step_bytes(cfg, L)[1] for L, _ in prof_L]
     attn_ms = float(np.mean(k_attn))
     achieved = float(np.mean(attn_b)) / (attn_ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "traffic": attn_traffic(cfg.B) if cfg.name == "llama" else None,
+            "kernel": "attn_kernel", "peak_kind": peak_kind, "bytes_per_launch": float(np.mean(attn_b))}
+    pcie = None
+    if cfg.offload:
+        # the step is bound by the slower of its HBM bytes at the HBM peak and its PCIe bytes
+        # at the UVA read ceiling; when PCIe is slower the gather kernel is the dominant one
+        t_hbm = float(np.mean(step_b)) / (hbm_peak * 1e9)
+        t_pcie = float(np.mean(pcie_b)) / (pcie_peak * 1e9)
+        gather_pcie = [step_bytes(cfg, L, int(misses[ti]))[3] for L, ti in prof_L]
+        g_ms = float(np.mean(k_gather))
+        pcie = {"bytes_per_step": float(np.mean(pcie_b)), "pages_per_step": float(np.mean([misses[ti] for _, ti in Ls])),
+                "step0_pages": int(misses[0]), "probe_gbs": pcie_peak,
+                "gather_gbs": float(np.mean(gather_pcie)) / (g_ms / 1e3) / 1e9 if g_ms > 0 else None,
+                "step_bound_us": 1e6 * max(t_hbm, t_pcie), "step_bound": "pcie" if t_pcie > t_hbm else "hbm",
+                "step_frac": 1e6 * max(t_hbm, t_pcie) / (1e3 * tot_ms / args.steps)}
+        if t_pcie > t_hbm and pcie["gather_gbs"]:
+            roof = {"bound": "pcie", "achieved": pcie["gather_gbs"], "peak": pcie_peak, "unit": "GB/s",
+                    "frac": pcie["gather_gbs"] / pcie_peak, "traffic": None, "kernel": "copy_kernel",
+                    "peak_kind": "measured (UVA read probe, this run)",
+                    "bytes_per_launch": float(np.mean(gather_pcie))}
     clocks = clk.summary()
     h2d = sum(x[0].numel() * x.element_size() for x in hp)
     d2h = o_host.numel() * 4 + s_host.numel() * 4 + m_host.numel() * 4
@@ -379,16 +458,15 @@ def run_gpu(args, cfg):
         "bytes_per_step": float(np.mean(step_b)),
         "kernel_us": {"score_select": 1e3 * float(np.mean(k_score)),
                       "gather": 1e3 * float(np.mean(k_gather)), "attention": 1e3 * attn_ms},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": attn_traffic(cfg.B) if cfg.name == "llama" else None,
-                     "kernel": "attn_kernel",
-                     "peak_kind": peak_kind,
-                     "bytes_per_launch": float(np.mean(attn_b))},
+        "roofline": roof,
+        "step0_us": 1e3 * step0_ms,
         "e2e": {"value": q_per_step / (e2e_ms / 1e3), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (3 if cfg.offload else 2),
         "clocks": clocks,
     }
+    if pcie is not None:
+        line["pcie"] = pcie
     if not args.no_cpu_baseline:
         cb, _ = oracle_sample(workload(args.workload, 4), 3, budget_s=args.cpu_budget)
         line["cpu_baseline"] = cb

@@ -213,6 +213,16 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
 nosa_status nosa_decode_attn_noalloc(const nosa_config* cfg, const nosa_state* st, const uint16_t* q,
                                      const int32_t* sel, float* out, void* stream);
 
+/*
+ * Measurement helper, not a step of the decode path (the pages give no such call): copies
+ * `bytes` of pinned, device-mapped host memory at `host` to device memory at `dev` with
+ * 16-byte loads over UVA, the access the gather kernel makes, on `ctas` CTAs of 256 threads
+ * (0: four per SM). The time of this call is the PCIe read ceiling the gather is measured
+ * against. host and dev must be 16-byte aligned and bytes a multiple of 16; NOSA_EINVAL
+ * otherwise, or when host is not pinned, device-mapped host memory. Asynchronous on stream.
+ */
+nosa_status nosa_uva_read_probe(const void* host, void* dev, size_t bytes, int ctas, void* stream);
+
 /* Synchronises the stream, reads state->err into *err_out (may be NULL):
  * NOSA_OK, NOSA_EDEVICE or NOSA_ETIMEOUT. */
 nosa_status nosa_check_device(const nosa_state* st, void* stream, uint32_t* err_out);

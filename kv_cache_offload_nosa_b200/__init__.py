@@ -25,7 +25,7 @@ ERR_BLOCK_TABLE, ERR_SEL, ERR_NO_VICTIM, ERR_TIMEOUT, ERR_FULL, ERR_INIT = 1, 2,
 EXPORTS = ("nosa_state_sizes", "nosa_workspace_size", "nosa_workspace_init", "nosa_state_init",
            "nosa_append", "nosa_score_blocks", "nosa_select", "nosa_gather", "nosa_decode_attn",
            "nosa_step", "nosa_check_device", "nosa_status_string", "nosa_last_error",
-           "nosa_decode_attn_noalloc")
+           "nosa_decode_attn_noalloc", "nosa_uva_read_probe")
 
 
 class nosa_config(ctypes.Structure):
@@ -79,6 +79,7 @@ def load(path: Optional[str] = None):
         "nosa_step": [cfgp, stp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp],
         "nosa_check_device": [stp, vp, ctypes.POINTER(ctypes.c_uint32)],
         "nosa_decode_attn_noalloc": [cfgp, stp, vp, vp, vp, vp],
+        "nosa_uva_read_probe": [vp, vp, sz, i32, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -188,6 +189,12 @@ def step(cfg, st, q, score_rows, k_new, v_new, evict, sel, out, miss_count, ws, 
     _check(load().nosa_step(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(score_rows),
                             _ptr(k_new), _ptr(v_new), _ptr(evict), _ptr(sel), _ptr(out),
                             _ptr(miss_count), _ptr(ws), ws_bytes, _stream(stream), ev))
+
+
+def uva_read_probe(host, dev, nbytes: int, ctas: int = 0, stream=None):
+    """Measurement helper: copies nbytes of pinned host memory to device memory by 16-byte UVA
+    loads (the gather's access); its time is the PCIe read ceiling of the gather."""
+    _check(load().nosa_uva_read_probe(_ptr(host), _ptr(dev), nbytes, ctas, _stream(stream)))
 
 
 def check_device(st, stream=None):

@@ -669,3 +669,50 @@ extern "C" nosa_status nosa_decode_attn_noalloc(const nosa_config* cfg, const no
   if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s);
   return launch_attn_t<64, 128>(c, a, tk, tv, s);
 }
+
+// ====================================================================== PCIe read ceiling
+// nosa_uva_read_probe: host -> device copy by 16-byte loads over UVA, four loads in flight
+// per thread, grid-stride. The gather kernel reads host pages the same way, so the probe's
+// rate is the ceiling the gather's achieved PCIe bandwidth is reported against.
+namespace {
+__global__ void __launch_bounds__(256) uva_read_kernel(const uint4* __restrict__ src,
+                                                       uint4* __restrict__ dst, size_t n) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n; i += 4 * stride) {
+    uint4 r[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) r[u] = src[i + u * stride];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) dst[i + u * stride] = r[u];
+  }
+  for (; i < n; i += stride) dst[i] = src[i];
+}
+}  // namespace
+
+extern "C" nosa_status nosa_uva_read_probe(const void* host, void* dev, size_t bytes, int ctas,
+                                           void* stream) {
+  NOSA_CHECK(host && dev, "host/dev is NULL");
+  NOSA_CHECK(aligned16(host) && aligned16(dev) && bytes % 16 == 0,
+             "host, dev and bytes must be multiples of 16");
+  NOSA_CHECK(ctas >= 0, "ctas < 0");
+  cudaPointerAttributes at;
+  cudaError_t e = cudaPointerGetAttributes(&at, host);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(NOSA_EINVAL, "host %p: %s", host, cudaGetErrorString(e));
+  }
+  NOSA_CHECK(at.type == cudaMemoryTypeHost && at.devicePointer == host,
+             "host %p is not pinned, device-mapped host memory", host);
+  if (bytes == 0) return NOSA_OK;
+  if (ctas == 0) {
+    int d = 0, sms = 0;
+    NOSA_CUDA(cudaGetDevice(&d));
+    NOSA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d));
+    ctas = 4 * sms;
+  }
+  uva_read_kernel<<<ctas, 256, 0, as_stream(stream)>>>(static_cast<const uint4*>(host),
+                                                       static_cast<uint4*>(dev), bytes / 16);
+  NOSA_CUDA(cudaGetLastError());
+  return NOSA_OK;
+}
