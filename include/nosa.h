@@ -202,8 +202,8 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
  * computes exactly what nosa_decode_attn computes but takes no workspace: its scratch (the
  * split-K partials and the per-group counters) lives in a static device array of 8 MiB
  * inside the library, which every GPU that loads the library keeps until the process exits.
- * Limit: B*Hkv * (8 * G * (d + 2) * 4 bytes, rounded up to 256) plus B*Hkv * 4 bytes must fit
- * in 8 MiB (about 500 groups at G = 4, d = 128); larger configurations get NOSA_ENOMEM and
+ * Limit: B*Hkv * (16 * G * (d + 2) * 4 bytes, rounded up to 256) plus B*Hkv * 4 bytes must
+ * fit in 8 MiB (about 250 groups at G = 4, d = 128); larger configurations get NOSA_ENOMEM and
  * must use nosa_decode_attn with a workspace. Allocates nothing: no cudaMalloc, no cudaFree.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress)
  * with that device current; make that first call before any stream capture. Every call

@@ -102,7 +102,8 @@ nosa_status check_state(const nosa_config& c, const nosa_state* st) {
 }
 
 struct WsLayout {
-  size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, ge_mask, sel_flag, total;
+  size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, ge_mask, sel_flag, copy_cnt,
+      copy_flag, total;
   int copy_stride;
 };
 
@@ -121,7 +122,9 @@ WsLayout ws_layout(const nosa_config& c) {
   w.copy_count = off; off += up256(NG * 4);
   w.partials = off; off += up256(NG * kPartialSlots * (size_t)G * (c.d + 2) * 4);
   w.ge_mask = off; off += up256(NG * (size_t)words(c) * 4);
-  w.sel_flag = off; off += up256(NG * 4);
+  w.sel_flag = off; off += up256(NG * kFlagStride * 4);
+  w.copy_cnt = off; off += up256(NG * 4);
+  w.copy_flag = off; off += up256(NG * kFlagStride * 4);
   w.total = off;
   return w;
 }
@@ -204,9 +207,27 @@ nosa_status launch_sel_kernel(void (*k)(StepArgs), const nosa_config& c, const S
   return NOSA_OK;
 }
 
-nosa_status launch_copy(const nosa_config& c, const nosa_state* st, void* ws, cudaStream_t s) {
+// CTAs of the flag-driven copy: 64 x 256 threads x 128 bytes in flight is about 2 MiB, well
+// above what PCIe needs to stay busy, while leaving the SMs to the score and attention CTAs.
+constexpr int kCopyCtas = 64;
+
+nosa_status launch_copy(const nosa_config& c, const nosa_state* st, void* ws, cudaStream_t s,
+                        bool flags = false) {
   const WsLayout w = ws_layout(c);
-  const int page_vec = c.block_size * c.d * 2 / 16;
+  CopyArgs ca;
+  ca.copy_list = ws_at<int2>(ws, w.copy_list);
+  ca.copy_stride = w.copy_stride;
+  ca.copy_count = ws_at<int32_t>(ws, w.copy_count);
+  ca.host_k = reinterpret_cast<const uint4*>(st->host_k);
+  ca.host_v = reinterpret_cast<const uint4*>(st->host_v);
+  ca.k_pool = reinterpret_cast<uint4*>(st->k_pool);
+  ca.v_pool = reinterpret_cast<uint4*>(st->v_pool);
+  ca.max_blocks = c.max_blocks;
+  ca.page_vec = c.block_size * c.d * 2 / 16;
+  ca.sel_flag = flags ? ws_at<uint32_t>(ws, w.sel_flag) : nullptr;
+  ca.copy_cnt = ws_at<uint32_t>(ws, w.copy_cnt);
+  ca.copy_flag = ws_at<uint32_t>(ws, w.copy_flag);
+  ca.err = st->err;
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(n_groups(c), 8);
   lc.blockDim = dim3(256);
@@ -216,12 +237,12 @@ nosa_status launch_copy(const nosa_config& c, const nosa_state* st, void* ws, cu
   at[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = at;
   lc.numAttrs = 1;
-  NOSA_CUDA(cudaLaunchKernelEx(&lc, copy_kernel, (const int2*)ws_at<int2>(ws, w.copy_list), w.copy_stride,
-                               (const int32_t*)ws_at<int32_t>(ws, w.copy_count),
-                               reinterpret_cast<const uint4*>(st->host_k),
-                               reinterpret_cast<const uint4*>(st->host_v),
-                               reinterpret_cast<uint4*>(st->k_pool), reinterpret_cast<uint4*>(st->v_pool),
-                               c.max_blocks, page_vec));
+  if (flags) {
+    lc.gridDim = dim3(kCopyCtas);
+    NOSA_CUDA(cudaLaunchKernelEx(&lc, copy_seq_kernel, ca, (int)n_groups(c)));
+  } else {
+    NOSA_CUDA(cudaLaunchKernelEx(&lc, copy_kernel, ca));
+  }
   return NOSA_OK;
 }
 
@@ -260,9 +281,12 @@ nosa_status make_pool_map(CUtensorMap* m, const nosa_config& c, void* pool) {
   return NOSA_OK;
 }
 
+// finest: the smallest split width the partial slots allow (used when the attention of each
+// group waits for that group's page copies: groups become ready one after another over the
+// whole PCIe transfer, so spreading each group over more CTAs shortens the last group's tail).
 template <int D, int BS>
 nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& tk, const CUtensorMap& tv,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool finest) {
   using SH = AttnShape<D, BS>;
   int stages = (110 * 1024) / SH::STAGE;
   stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
@@ -279,6 +303,7 @@ nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& t
   const long long target = (long long)sms * per_sm;
   const int wmin = (a.k + kPartialSlots - 2) / (kPartialSlots - 1);
   int W = c.attn_split;
+  if (W <= 0 && finest) W = wmin;
   if (W <= 0) {
     // Prefer a divisor of k: every CTA then holds one segment of one group and never flushes
     // in mid-stream. Aim at about two CTAs per resident slot (finer work overlaps the
@@ -312,8 +337,10 @@ nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& t
   return NOSA_OK;
 }
 
+// ready: per-group flags the attention waits on (and clears), or NULL to wait for the
+// previous grid as a whole.
 nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16_t* q, const int32_t* sel,
-                        float* out, void* ws, cudaStream_t s, bool flags = false) {
+                        float* out, void* ws, cudaStream_t s, uint32_t* ready = nullptr) {
   CUtensorMap tk, tv;
   nosa_status r = make_pool_map(&tk, c, st->k_pool);
   if (r != NOSA_OK) return r;
@@ -338,15 +365,16 @@ nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16
   a.total = n_groups(c) * kk(c);
   a.total_pages = (long long)n_groups(c) * c.slots;
   a.scale_log2 = c.scale * 1.4426950408889634f;
-  a.sel_flag = flags ? ws_at<uint32_t>(ws, w.sel_flag) : nullptr;
+  a.sel_flag = ready;
+  const bool finest = ready != nullptr && has_host(st);
   if (c.d == 128) {
-    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s);
-    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s);
-    return launch_attn_t<128, 128>(c, a, tk, tv, s);
+    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s, finest);
+    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s, finest);
+    return launch_attn_t<128, 128>(c, a, tk, tv, s, finest);
   }
-  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s);
-  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s);
-  return launch_attn_t<64, 128>(c, a, tk, tv, s);
+  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s, finest);
+  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s, finest);
+  return launch_attn_t<64, 128>(c, a, tk, tv, s, finest);
 }
 
 }  // namespace
@@ -555,15 +583,20 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   a.evict = evict;
   a.sel = sel;
   a.miss_count = miss_count;
-  // Without host pools the attention starts on each group as soon as that group's selection
-  // is published (per-group flags); with host pools it waits for the page copies.
-  const bool flags = !has_host(st) && !events;
-  a.sel_flag = flags ? ws_at<uint32_t>(ws, ws_layout(c).sel_flag) : nullptr;
+  // Per-group flags chain the kernels group by group: the attention of a group starts as soon
+  // as that group's selection is published or, with host pools, as soon as its page copies
+  // (which themselves start on the group's published plan) have landed. With events each
+  // kernel waits for the previous one as a whole, so that the events time kernels alone.
+  const WsLayout w = ws_layout(c);
+  const bool flags = !events;
+  a.sel_flag = flags ? ws_at<uint32_t>(ws, w.sel_flag) : nullptr;
+  uint32_t* ready = !flags ? nullptr
+                           : ws_at<uint32_t>(ws, has_host(st) ? w.copy_flag : w.sel_flag);
   if ((r = launch_score<true>(c, a, s)) != NOSA_OK) return r;
   if ((r = rec(1)) != NOSA_OK) return r;
-  if (has_host(st) && (r = launch_copy(c, st, ws, s)) != NOSA_OK) return r;
+  if (has_host(st) && (r = launch_copy(c, st, ws, s, flags)) != NOSA_OK) return r;
   if ((r = rec(2)) != NOSA_OK) return r;
-  if ((r = launch_attn(c, st, q, sel, out, ws, s, flags)) != NOSA_OK) return r;
+  if ((r = launch_attn(c, st, q, sel, out, ws, s, ready)) != NOSA_OK) return r;
   return rec(3);
 }
 
@@ -660,14 +693,15 @@ extern "C" nosa_status nosa_decode_attn_noalloc(const nosa_config* cfg, const no
   a.total = n_groups(c) * kk(c);
   a.total_pages = (long long)n_groups(c) * c.slots;
   a.scale_log2 = c.scale * 1.4426950408889634f;
+  const bool finest = false;
   if (c.d == 128) {
-    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s);
-    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s);
-    return launch_attn_t<128, 128>(c, a, tk, tv, s);
+    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s, finest);
+    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s, finest);
+    return launch_attn_t<128, 128>(c, a, tk, tv, s, finest);
   }
-  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s);
-  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s);
-  return launch_attn_t<64, 128>(c, a, tk, tv, s);
+  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s, finest);
+  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s, finest);
+  return launch_attn_t<64, 128>(c, a, tk, tv, s, finest);
 }
 
 // ====================================================================== PCIe read ceiling

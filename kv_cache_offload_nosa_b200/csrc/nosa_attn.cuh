@@ -42,7 +42,7 @@ struct AttnArgs {
   int stages;
   long long total_pages;
   float scale_log2;           // sigma * log2(e)
-  uint32_t* sel_flag;         // [B*Hkv] per-group "selection published" flags, or NULL
+  uint32_t* sel_flag;         // [B*Hkv * kFlagStride] per-group "ready" flags, or NULL
 };
 
 struct TaskInfo {
@@ -119,10 +119,19 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
     for (int base = 0; base < ntask && !abort; base += 32) {
       const int i_l = base + lane;
       int gi_l = 0, j_l = -1, L_l = 0, page_l = -1;
+      if (flags) {
+        // lane 0 acquires the flags of the batch's groups (contiguous, in order); the warp
+        // barrier orders the other lanes' loads below (L2, __ldcg) after those acquires
+        if (lane == 0) {
+          const int g1 = (task0 + min(base + 32, ntask) - 1) / a.k;
+          for (int g = (task0 + base) / a.k; g <= g1; ++g)
+            if (!wait_flag(a.sel_flag + (size_t)g * kFlagStride, deadline)) set_err(a.err, NOSA_ERR_TIMEOUT);
+        }
+        __syncwarp();
+      }
       if (i_l < ntask) {
         const int t = task0 + i_l;
         gi_l = t / a.k;
-        if (flags && !wait_flag(a.sel_flag + gi_l, deadline)) set_err(a.err, NOSA_ERR_TIMEOUT);
         L_l = __ldcg(a.seq_len + gi_l);
         const int N = (L_l + BS - 1) / BS;
         j_l = __ldcg(a.sel + t);
@@ -378,7 +387,7 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
         }
         if (tid == 0) {
           a.counters[gi] = 0u;
-          if (flags) a.sel_flag[gi] = 0u;  // every CTA of this group has passed its wait
+          if (flags) a.sel_flag[(size_t)gi * kFlagStride] = 0u;  // every CTA of the group passed its wait
         }
       }
       named_bar(1, NC * 32);

@@ -13,7 +13,10 @@ namespace nosa {
 
 constexpr int kMaxBlocks = 8192;           // per group (selection keys live in shared memory)
 constexpr int kMaxWords = kMaxBlocks / 32;
-constexpr int kPartialSlots = 8;           // split-K segments per group
+constexpr int kPartialSlots = 16;          // split-K segments per group
+// Per-group flags sit 128 bytes apart (one cache line each): waiters of different groups
+// poll different lines, so no single L2 slice takes every poll.
+constexpr int kFlagStride = 32;            // uint32 words between consecutive groups' flags
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // bounded spin: 4 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

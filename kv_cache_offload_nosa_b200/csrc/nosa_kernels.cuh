@@ -49,7 +49,7 @@ struct StepArgs {
   int32_t* miss_count;
   uint32_t* counters;
   uint32_t* ge_mask;      // [B*Hkv][W] Gamma_e handed from chunk 0 to the last chunk
-  uint32_t* sel_flag;     // [B*Hkv] set (release) once a group's selection is published, or NULL
+  uint32_t* sel_flag;     // [B*Hkv * kFlagStride] set (release) once a group's selection is published, or NULL
   uint32_t* err;
 };
 
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
     __syncthreads();
     if (tid == 0) {
       __threadfence();
-      st_release_gpu(a.sel_flag + gi, 1u);
+      st_release_gpu(a.sel_flag + (size_t)gi * kFlagStride, 1u);
     }
   }
 }
@@ -305,36 +305,102 @@ __global__ void __launch_bounds__(kSelThreads) plan_kernel(StepArgs a) {
 }
 
 // Host -> HBM page copies over UVA (pinned host memory read by the kernel with 16-byte
-// loads; NOSA's "Comunicacion de Alto Ancho de Banda"). grid = (groups, CTAs per group).
-__global__ void __launch_bounds__(256) copy_kernel(const int2* copy_list, int copy_stride,
-                                                   const int32_t* copy_count, const uint4* host_k,
-                                                   const uint4* host_v, uint4* k_pool, uint4* v_pool,
-                                                   int max_blocks, int page_vec) {
+// loads; NOSA's "Comunicacion de Alto Ancho de Banda"). copy_kernel: grid = (groups, CTAs per
+// group), after the whole previous grid; copy_seq_kernel below: the flag-driven form.
+struct CopyArgs {
+  const int2* copy_list;
+  int copy_stride;
+  const int32_t* copy_count;
+  const uint4* host_k;
+  const uint4* host_v;
+  uint4* k_pool;
+  uint4* v_pool;
+  int max_blocks, page_vec;
+  uint32_t* sel_flag;    // [groups * kFlagStride] plan published (copy_seq_kernel)
+  uint32_t* copy_cnt;    // [groups] CTAs done with the group (copy_seq_kernel; starts, ends at 0)
+  uint32_t* copy_flag;   // [groups * kFlagStride] pages in place (copy_seq_kernel)
+  uint32_t* err;
+};
+
+__global__ void __launch_bounds__(256) copy_kernel(CopyArgs a) {
   griddep_wait();
   griddep_launch_dependents();
   const int gi = blockIdx.x;
-  const int n = copy_count[gi];
+  const int n = __ldcg(a.copy_count + gi);
   for (int i = blockIdx.y; i < n; i += gridDim.y) {
-    const int2 e = copy_list[(size_t)gi * copy_stride + i];
-    const size_t src = ((size_t)gi * max_blocks + e.x) * page_vec;
-    const size_t dst = (size_t)e.y * page_vec;
-    for (int v0 = threadIdx.x; v0 < page_vec; v0 += 4 * blockDim.x) {
+    const int2 e = __ldcg(a.copy_list + (size_t)gi * a.copy_stride + i);
+    const size_t src = ((size_t)gi * a.max_blocks + e.x) * a.page_vec;
+    const size_t dst = (size_t)e.y * a.page_vec;
+    for (int v0 = threadIdx.x; v0 < a.page_vec; v0 += 4 * blockDim.x) {
       uint4 rk[4], rv[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int v = v0 + u * blockDim.x;
-        if (v < page_vec) {
-          rk[u] = host_k[src + v];
-          rv[u] = host_v[src + v];
+        if (v < a.page_vec) {
+          rk[u] = a.host_k[src + v];
+          rv[u] = a.host_v[src + v];
         }
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int v = v0 + u * blockDim.x;
-        if (v < page_vec) {
-          k_pool[dst + v] = rk[u];
-          v_pool[dst + v] = rv[u];
+        if (v < a.page_vec) {
+          a.k_pool[dst + v] = rk[u];
+          a.v_pool[dst + v] = rv[u];
         }
+      }
+    }
+  }
+}
+
+// Flag-driven form of the copy: a pool of CTAs walks the groups in order and shares each
+// group's pages among its CTAs (one block, K and V page, per CTA at a time). PCIe stays busy
+// from the first published plan on, and the pages of group g land before those of g + 1, so
+// the attention of the early groups overlaps the transfers of the later ones. The CTA that
+// finishes a group last publishes copy_flag (and clears the group's sel_flag and counter).
+__global__ void __launch_bounds__(256) copy_seq_kernel(CopyArgs a, int ngroups) {
+  griddep_launch_dependents();
+  __shared__ int s_n;
+  const unsigned long long deadline = globaltimer() + kWaitLimitNs;
+  for (int gi = 0; gi < ngroups; ++gi) {
+    if (threadIdx.x == 0) {
+      if (!wait_flag(a.sel_flag + (size_t)gi * kFlagStride, deadline)) set_err(a.err, NOSA_ERR_TIMEOUT);
+      s_n = __ldcg(a.copy_count + gi);
+    }
+    __syncthreads();
+    const int n = s_n;
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+      const int2 e = __ldcg(a.copy_list + (size_t)gi * a.copy_stride + i);
+      const size_t src = ((size_t)gi * a.max_blocks + e.x) * a.page_vec;
+      const size_t dst = (size_t)e.y * a.page_vec;
+      for (int v0 = threadIdx.x; v0 < a.page_vec; v0 += 4 * blockDim.x) {
+        uint4 rk[4], rv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int v = v0 + u * blockDim.x;
+          if (v < a.page_vec) {
+            rk[u] = a.host_k[src + v];
+            rv[u] = a.host_v[src + v];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int v = v0 + u * blockDim.x;
+          if (v < a.page_vec) {
+            a.k_pool[dst + v] = rk[u];
+            a.v_pool[dst + v] = rv[u];
+          }
+        }
+      }
+    }
+    __syncthreads();  // s_n is rewritten for the next group only after every thread read it
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(a.copy_cnt + gi, 1u) == gridDim.x - 1) {
+        a.copy_cnt[gi] = 0u;
+        a.sel_flag[(size_t)gi * kFlagStride] = 0u;
+        __threadfence();
+        st_release_gpu(a.copy_flag + (size_t)gi * kFlagStride, 1u);
       }
     }
   }

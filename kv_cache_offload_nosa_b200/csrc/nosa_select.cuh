@@ -185,15 +185,16 @@ struct KeyBuckets {
 
 // Top-m of key[] over the candidate bitmask cand[0..W): higher key first, equal keys to
 // the lower index. Writes the bitmask into out[0..W). Returns min(m, |cand|).
-// All threads of the CTA must call it; W <= blockDim.x. float_keys: the keys are ord_f32
-// images of floats.
+// All threads of the CTA must call it; W <= blockDim.x. FLOAT_KEYS: the keys are ord_f32
+// images of floats (scores); otherwise they may tie massively (LRU stamps), and the
+// histogram, the boundary list and an all-equal boundary bucket are handled for that.
 //  1. one pass: candidate count, smallest and largest key;
 //  2. keys fall into 256 buckets spanning [min, max] (KeyBuckets), a histogram finds the
 //     bucket holding the m-th key;
 //  3. buckets above it are taken whole; the boundary bucket's keys are ranked exactly
 //     against each other (or, if it holds more than kSmallSel keys, radix-selected).
-__device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, int W, int m,
-                        bool float_keys) {
+template <bool FLOAT_KEYS>
+__device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, int W, int m) {
   const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int nw = nth >> 5;
   const int span = W * 32;
@@ -234,9 +235,27 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
     __syncthreads();
     return m <= 0 ? 0 : total;
   }
-  const KeyBuckets bucket(kmin, kmax, float_keys);
-  for (int j = tid; j < span; j += nth)
-    if ((cand[j >> 5] >> (j & 31)) & 1u) atomicAdd(&S.hist[bucket(S.key[j])], 1);
+  const KeyBuckets bucket(kmin, kmax, FLOAT_KEYS);
+  // histogram. Scores spread over the buckets and plain atomics rarely collide; other keys
+  // (e.g. blocks last used at the same step) can pile into one bucket, so there a warp
+  // whose keys share one bucket adds them with a single atomic.
+  if constexpr (FLOAT_KEYS) {
+    for (int j = tid; j < span; j += nth)
+      if ((cand[j >> 5] >> (j & 31)) & 1u) atomicAdd(&S.hist[bucket(S.key[j])], 1);
+  } else for (int j = tid; j < span; j += nth) {  // span is a multiple of 32: warp-uniform
+    const bool in = (cand[j >> 5] >> (j & 31)) & 1u;
+    const uint32_t bk = in ? bucket(S.key[j]) : 0u;
+    const unsigned act = __ballot_sync(0xffffffffu, in);
+    if (act) {
+      const int lead = __ffs(act) - 1;
+      const uint32_t b0 = __shfl_sync(0xffffffffu, bk, lead);
+      if (__all_sync(0xffffffffu, !in || bk == b0)) {
+        if (lane == lead) atomicAdd(&S.hist[b0], __popc(act));
+      } else if (in) {
+        atomicAdd(&S.hist[bk], 1);
+      }
+    }
+  }
   __syncthreads();
   if (tid < 32) {
     int c[8], sum = 0;
@@ -273,12 +292,13 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
   for (int base = 0; base < span; base += nth) {
     const int j = base + tid;
     bool take = false, bnd = false;
+    uint32_t k = 0u;
     if (j < span && ((cand[j >> 5] >> (j & 31)) & 1u)) {
-      const uint32_t k = S.key[j];
+      k = S.key[j];
       const uint32_t bk = bucket(k);
       take = bk > bstar;
       bnd = bk == bstar;
-      if (bnd && small) {
+      if (FLOAT_KEYS && bnd && small) {
         const int slot = atomicAdd(&S.sc[2], 1);
         S.list[slot] = j;
         S.lkey[slot] = k;
@@ -286,6 +306,18 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
     }
     const uint32_t tw = __ballot_sync(0xffffffffu, take);
     const uint32_t bw = __ballot_sync(0xffffffffu, bnd);
+    if (!FLOAT_KEYS && small && bw) {
+      // tied keys: one atomic per warp reserves the warp's slots in the boundary list
+      const int lead = __ffs(bw) - 1;
+      int slot0 = 0;
+      if (lane == lead) slot0 = atomicAdd(&S.sc[2], __popc(bw));
+      slot0 = __shfl_sync(0xffffffffu, slot0, lead);
+      if (bnd) {
+        const int slot = slot0 + __popc(bw & ((1u << lane) - 1u));
+        S.list[slot] = j;
+        S.lkey[slot] = k;
+      }
+    }
     if (lane == 0 && j < span) {
       out[j >> 5] = tw;
       if (!small) S.m2[j >> 5] = bw;
@@ -305,8 +337,52 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
       if (rank < rem) atomicOr(&out[j >> 5], 1u << (j & 31));
     }
     __syncthreads();
-  } else {
+  } else if constexpr (FLOAT_KEYS) {
     sel_topm_radix(S, S.m2, out, W, rem);
+  } else {
+    // The boundary bucket is too large to rank key against key. When all its keys are equal
+    // (blocks last used at the same step) the lowest indices win, and a prefix count over
+    // the bucket's mask words decides; otherwise radix select.
+    uint32_t bmin = 0xffffffffu, bmax = 0u;
+    for (int j = tid; j < span; j += nth) {
+      if ((S.m2[j >> 5] >> (j & 31)) & 1u) {
+        const uint32_t k = S.key[j];
+        bmin = min(bmin, k);
+        bmax = max(bmax, k);
+      }
+    }
+    bmin = __reduce_min_sync(0xffffffffu, bmin);
+    bmax = __reduce_max_sync(0xffffffffu, bmax);
+    if (lane == 0) {
+      ured[warp] = bmin;
+      ured[8 + warp] = bmax;
+    }
+    __syncthreads();
+    bmin = 0xffffffffu;
+    bmax = 0u;
+    for (int i = 0; i < nw; ++i) {
+      bmin = min(bmin, ured[i]);
+      bmax = max(bmax, ured[8 + i]);
+    }
+    __syncthreads();  // ured is reused by the scan below
+    if (bmin == bmax) {
+      const uint32_t bw = (tid < W) ? S.m2[tid] : 0u;
+      const int before = block_exclusive_scan(__popc(bw), S.red, nullptr);
+      if (tid < W) {
+        int take = rem - before;
+        take = take < 0 ? 0 : (take > __popc(bw) ? __popc(bw) : take);
+        uint32_t t = bw, keep = 0u;
+        for (int x = 0; x < take; ++x) {
+          const uint32_t low = t & (~t + 1u);
+          keep |= low;
+          t ^= low;
+        }
+        out[tid] |= keep;
+      }
+      __syncthreads();
+    } else {
+      sel_topm_radix(S, S.m2, out, W, rem);
+    }
   }
   return m;
 }
@@ -369,7 +445,7 @@ __device__ int select_evict(const SelSmem& S, const float* evict, const uint32_t
     S.cand[w] = prev[w] & a & word_valid_mask(w, N);
   }
   __syncthreads();
-  const int ne = sel_topm(S, S.cand, S.ge, W, k_e, true);
+  const int ne = sel_topm<true>(S, S.cand, S.ge, W, k_e);
   for (int w = tid; w < Wmax; w += nth) {
     const uint32_t c = (w < W) ? S.cand[w] : 0u;
     const uint32_t g = (w < W) ? S.ge[w] : 0u;
@@ -404,7 +480,7 @@ __device__ void select_query(const SelSmem& S, const float* scores, const uint32
   for (int i = 0; i < (nth >> 5); ++i) ne += S.red[i];
   __syncthreads();
   const int mq = (k - ne < N - ne) ? k - ne : N - ne;
-  sel_topm(S, S.cand, S.pick, W, mq, true);
+  sel_topm<true>(S, S.cand, S.pick, W, mq);
   for (int w = tid; w < Wmax; w += nth) {
     const uint32_t s = (w < W) ? (S.ge[w] | S.pick[w]) : 0u;
     S.sset[w] = s;
@@ -449,23 +525,37 @@ __device__ void plan_group(const SelSmem& S, const PlanArgs& p) {
   const int W = (N + 31) / 32;
   const int tail = (p.L - 1) / p.bs;
   const int Wf = (p.slots + 31) / 32;
-  // need (m1), resident (m2)
-  if (tid < W) {
-    uint32_t need = S.sset[tid];
-    if ((tail >> 5) == tid) need |= 1u << (tail & 31);
-    uint32_t res = 0;
-    for (int b = 0; b < 32; ++b) {
-      const int j = tid * 32 + b;
-      if (j >= N) break;
-      const int pg = p.block_table[j];
-      if (pg >= 0) {
-        if (pg < p.page_base || pg >= p.page_base + p.slots) set_err(p.err, NOSA_ERR_BLOCK_TABLE);
-        else res |= 1u << b;
+  // need (m1), resident (m2), misses (cand). Global tables are read element-strided, one
+  // entry per thread, and each warp assembles one 32-bit word per pass with a ballot: all
+  // loads of a pass are in flight together instead of one dependent load per block.
+  const int lane = tid & 31, warp = tid >> 5;
+  constexpr int U = 8;  // loads in flight per thread
+  for (int j00 = 0; j00 < W * 32; j00 += U * nth) {
+    int pg[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j00 + u * nth + tid;
+      pg[u] = (j < N) ? p.block_table[j] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j0 = j00 + u * nth;
+      if (j0 >= W * 32) break;
+      bool res = false;
+      if (pg[u] >= 0) {
+        if (pg[u] < p.page_base || pg[u] >= p.page_base + p.slots) set_err(p.err, NOSA_ERR_BLOCK_TABLE);
+        else res = true;
+      }
+      const uint32_t rw = __ballot_sync(0xffffffffu, res);
+      const int w = (j0 >> 5) + warp;
+      if (lane == 0 && w < W) {
+        uint32_t need = S.sset[w];
+        if ((tail >> 5) == w) need |= 1u << (tail & 31);
+        S.m1[w] = need;
+        S.m2[w] = rw;
+        S.cand[w] = need & ~rw;
       }
     }
-    S.m1[tid] = need;
-    S.m2[tid] = res;
-    S.cand[tid] = need & ~res;  // misses
   }
   __syncthreads();
   int nmiss = 0;
@@ -473,14 +563,23 @@ __device__ void plan_group(const SelSmem& S, const PlanArgs& p) {
   const int nm = block_sum(nmiss, S.red);
   // free slots -> pick (bitmask over slots)
   int nfr = 0;
-  for (int w = tid; w < Wf; w += nth) {
-    uint32_t f = 0;
-    for (int b = 0; b < 32; ++b) {
-      const int z = w * 32 + b;
-      if (z < p.slots && p.slot_owner[z] < 0) f |= 1u << b;
+  for (int z00 = 0; z00 < Wf * 32; z00 += U * nth) {
+    int ow[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int z = z00 + u * nth + tid;
+      ow[u] = (z < p.slots) ? p.slot_owner[z] : 0;
     }
-    S.pick[w] = f;
-    nfr += __popc(f);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int z0 = z00 + u * nth;
+      if (z0 >= Wf * 32) break;
+      const bool f = ow[u] < 0;
+      const uint32_t fw = __ballot_sync(0xffffffffu, f);
+      const int w = (z0 >> 5) + warp;
+      if (lane == 0 && w < Wf) S.pick[w] = fw;
+      nfr += f ? 1 : 0;
+    }
   }
   const int nfree = block_sum(nfr, S.red);
   const int nf_use = nm < nfree ? nm : nfree;
@@ -488,13 +587,22 @@ __device__ void plan_group(const SelSmem& S, const PlanArgs& p) {
   // victims -> ge (reused as the victim bitmask)
   if (nv > 0) {
     if (tid < W) S.m2[tid] = S.m2[tid] & ~S.m1[tid];  // evictable
-    for (int w = tid; w < W; w += nth) {
-      const uint32_t v = S.m2[w];
-      for (int b = 0; b < 32; ++b)
-        if ((v >> b) & 1u) S.key[w * 32 + b] = ord_lru(p.last_used[w * 32 + b]);
+    __syncthreads();
+    for (int j00 = 0; j00 < W * 32; j00 += U * nth) {
+      int lu[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j00 + u * nth + tid;
+        lu[u] = (j < W * 32 && ((S.m2[j >> 5] >> (j & 31)) & 1u)) ? p.last_used[j] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j00 + u * nth + tid;
+        if (j < W * 32 && ((S.m2[j >> 5] >> (j & 31)) & 1u)) S.key[j] = ord_lru(lu[u]);
+      }
     }
     __syncthreads();
-    const int got = sel_topm(S, S.m2, S.ge, W, nv, false);
+    const int got = sel_topm<false>(S, S.m2, S.ge, W, nv);
     if (got < nv) {
       set_err(p.err, NOSA_ERR_NO_VICTIM);
       nv = got;
@@ -552,10 +660,9 @@ __device__ void plan_group(const SelSmem& S, const PlanArgs& p) {
         }
         ++r;
       }
-      const uint32_t need = S.m1[tid];
-      for (int b = 0; b < 32; ++b)
-        if ((need >> b) & 1u) p.last_used[tid * 32 + b] = p.L;
     }
+    for (int j = tid; j < W * 32; j += nth)
+      if ((S.m1[j >> 5] >> (j & 31)) & 1u) p.last_used[j] = p.L;
     if (tid == 0) {
       *p.copy_count = nassign;
       if (p.miss_count) *p.miss_count = nm;
