@@ -475,6 +475,131 @@ def run_gpu(args, cfg):
         dist.destroy_process_group()
 
 
+# ----------------------------------------------------------------------------- lookahead
+def run_lookahead(args, cfg):
+    """Tokens through `--layers` offload layers (independent caches of the workload's shape):
+    SparDA's lookahead pipeline (plans ahead, layer-ordered copies on their own stream,
+    attention after each layer's copies) against the same layers stepped one after another
+    with nosa_step. Reports both token times and the time the pipeline hides."""
+    import torch
+    import kv_cache_offload_nosa_b200 as nosa
+    from kv_cache_offload_nosa_b200 import build as nb
+    from kv_cache_offload_nosa_b200 import dist as D
+    from kv_cache_offload_nosa_b200.lookahead import LookaheadPipeline
+
+    rank, world, local = D.rank_info()
+    torch.cuda.set_device(local)
+    D.init("nccl", timeout_s=300)
+    nb.build()
+    nl = args.layers
+    total = 2 * (args.warmup + args.steps)
+    cfgs = [cfg.with_(cfg_id=cfg.cfg_id + 1000 * l + 100000 * rank, steps=total) for l in range(nl)]
+    NG = cfg.B * cfg.Hkv
+    caches, ins = [], []
+    for c in cfgs:
+        inp = syn.make_inputs(c)
+        cc = nosa.make_config(c.B, c.Hq, c.Hkv, c.d, c.block, c.sub_block, c.k_q, c.k_e, c.max_blocks,
+                              slots=c.n_slots, n_score_rows=c.rows, scale=c.scale)
+        cache = nosa.NosaCache(cc, offload=True)
+        cache.pool_view("host_k").copy_(torch.from_numpy(inp.pool_k.reshape(NG, c.max_blocks, c.block, c.d)).view(torch.int16))
+        cache.pool_view("host_v").copy_(torch.from_numpy(inp.pool_v.reshape(NG, c.max_blocks, c.block, c.d)).view(torch.int16))
+        inp.pool_k = inp.pool_v = None
+        cache.init(torch.tensor(c.T, dtype=torch.int32, device="cuda"),
+                   torch.from_numpy(inp.resident.reshape(NG, -1)).cuda())
+        zero = np.zeros((c.B, c.Hkv), np.int64)
+        qs, prev = [], None
+        for t in range(total):
+            prev = syn.query_step(c, t, prev, zero)
+            qs.append(syn.round_bf16(prev))
+        fc = np.stack([syn.round_bf16(syn.forecast_step(c, t, zero)) for t in range(total)])
+        ins.append({"q": torch.from_numpy(np.stack(qs)).view(torch.int16).cuda(),
+                    "f": torch.from_numpy(fc).view(torch.int16).cuda(),
+                    "kn": torch.from_numpy(inp.k_new).view(torch.int16).cuda(),
+                    "vn": torch.from_numpy(inp.v_new).view(torch.int16).cuda(),
+                    "ev": torch.from_numpy(inp.evict).cuda()})
+        caches.append(cache)
+    sel = [torch.empty(NG * cfg.k, dtype=torch.int32, device="cuda") for _ in range(nl)]
+    out = [torch.empty(cfg.B * cfg.Hq * cfg.d, dtype=torch.float32, device="cuda") for _ in range(nl)]
+    miss = torch.zeros((total, nl, -(-NG // 4) * 4), dtype=torch.int32, device="cuda")
+    flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush_sink = torch.empty((), dtype=torch.float32, device="cuda")
+    pipe = LookaheadPipeline(caches)
+    stream = torch.cuda.current_stream()
+
+    def pipelined(t):
+        pipe.token([x["f"][t] for x in ins], [x["ev"][t] for x in ins], [x["q"][t] for x in ins],
+                   [x["kn"][t] for x in ins], [x["vn"][t] for x in ins], sel,
+                   [miss[t, l, :NG] for l in range(nl)], out, stream=stream)
+
+    def serial(t):
+        for l, (c, x) in enumerate(zip(caches, ins)):
+            c.step(x["q"][t], x["kn"][t], x["vn"][t], x["ev"][t], sel[l], out[l], miss[t, l, :NG],
+                   score_rows=x["f"][t], stream=stream)
+
+    def timed(fn, t0, n):
+        ms = []
+        for i in range(n):
+            flush_w.zero_()
+            torch.sum(flush_r, dim=0, out=flush_sink)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn(t0 + i)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        return ms
+
+    t = 0
+    timed(pipelined, t, args.warmup)
+    t += args.warmup
+    D.barrier()
+    with Clocks(local) as clk:
+        pipe_ms = timed(pipelined, t, args.steps)
+    t += args.steps
+    pipe_misses = miss[t - args.steps:t].sum().item()
+    timed(serial, t, args.warmup)
+    t += args.warmup
+    ser_ms = timed(serial, t, args.steps)
+    ser_misses = miss[t - args.steps:t].sum().item()
+    for c in caches:
+        rc, err = c.check()
+        if rc != 0:
+            raise RuntimeError(f"device fault: rc={rc} err={err}")
+    pcie_peak = pcie_ceiling(nosa, torch)
+    tok_ms, ser_tok_ms = D.max_over_ranks([float(np.sum(pipe_ms)), float(np.sum(ser_ms))], device="cuda")
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    tok = tok_ms / args.steps
+    ser = ser_tok_ms / args.steps
+    page = cfg.block * cfg.d * 2
+    pcie_tok = pipe_misses / args.steps * 2 * page      # bytes per token (all layers)
+    q_tok = cfg.B * cfg.Hq * nl * world
+    line = {
+        "metric": METRIC, "value": q_tok / (tok / 1e3), "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tok / nl, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(cfg) + f" x {nl} layers, lookahead pipeline (forecast row per group)",
+                   "global_batch": cfg.B * world, "seq_len": cfg.T[0], "layers": nl,
+                   "parallelism": f"replicas x{world} (batch-sharded, no collective)",
+                   "l2": "flushed before every timed token (256 MiB write, then 256 MiB read)"},
+        "token_us": 1e3 * tok, "serial_token_us": 1e3 * ser, "hidden_us": 1e3 * (ser - tok),
+        "speedup_vs_serial": ser / tok,
+        "pcie": {"bytes_per_token": pcie_tok, "probe_gbs": pcie_peak,
+                 "bound_token_us": 1e6 * pcie_tok / (pcie_peak * 1e9),
+                 "frac": 1e6 * pcie_tok / (pcie_peak * 1e9) / (1e3 * tok),
+                 "serial_pages_per_token": ser_misses / args.steps,
+                 "pipelined_pages_per_token": pipe_misses / args.steps},
+        "gpu_launches": args.steps * nl * 4,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -486,12 +611,15 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=4, help="layers of the lookahead workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = workload(args.workload, args.warmup + args.steps, args.batch)
     if args.impl == "reference":
         run_reference(args, cfg)
+    elif cfg.name == "lookahead" and args.impl == "native":
+        run_lookahead(args, cfg)
     else:
         run_gpu(args, cfg)
 

@@ -195,6 +195,41 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
                       void* workspace, size_t ws_bytes, void* stream, void* const* events);
 
 /*
+ * Lookahead decoding (SparDA, gist.science/de/paper/2606.04511, section 2: "Trainierbare
+ * Lookahead Sparse-Selektion", "Asynchrones Prefetching mit persistentem UVA-Kernel"): the
+ * blocks a step attends are chosen from a forecast row before the step's query exists, so
+ * their host -> HBM copies can run while other work (e.g. the previous layer) computes.
+ * Three calls per step and state, in this order:
+ *
+ * nosa_plan_ahead scores the cache as it stands (no append) with score_rows
+ * ([B*Hkv][n_score_rows][d] bf16, e.g. one forecast row per group), runs the dual selection
+ * (sel [B*Hkv][k] and miss_count [B*Hkv] as in nosa_step) and, with host pools, the
+ * residency plan.
+ *
+ * nosa_prefetch (host pools; a no-op without) copies the planned pages host -> HBM over UVA,
+ * group after group. It may run on another stream once nosa_plan_ahead has completed.
+ *
+ * nosa_attend appends k_new / v_new ([B*Hkv][d] bf16) and attends q ([B][Hq][d] bf16) over
+ * the blocks sel chose (out [B][Hq][d] fp32). On the GPU each group first acquires its
+ * "pages in place" flag (bounded wait, NOSA_ERR_TIMEOUT on expiry). It must be issued after
+ * nosa_plan_ahead has completed; issue it after nosa_prefetch has completed too (same
+ * stream, or an event), so that its CTAs never sit on the SMs waiting for copies.
+ *
+ * Rules: the three calls of a step use the same state, workspace and sel, and no other call
+ * on that state and workspace comes between them. The triple computes what the oracle's
+ * lookahead order defines: select and plan at length L, append (L + 1), attend; a block the
+ * append creates is not a candidate of the step. Needs a non-empty cache (L >= 1).
+ */
+nosa_status nosa_plan_ahead(const nosa_config* cfg, const nosa_state* st, const uint16_t* score_rows,
+                            const float* evict, int32_t* sel, int32_t* miss_count, void* workspace,
+                            size_t ws_bytes, void* stream);
+nosa_status nosa_prefetch(const nosa_config* cfg, const nosa_state* st, void* workspace, size_t ws_bytes,
+                          void* stream);
+nosa_status nosa_attend(const nosa_config* cfg, const nosa_state* st, const uint16_t* q,
+                        const uint16_t* k_new, const uint16_t* v_new, const int32_t* sel, float* out,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * No-allocation variant of nosa_decode_attn (the pages have no counterpart: this is an
  * integration aid). Some callers cannot call cudaMalloc when they run attention: code being
  * captured into a CUDA graph, plugins inside a host framework that owns all device memory,

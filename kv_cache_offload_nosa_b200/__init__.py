@@ -25,7 +25,7 @@ ERR_BLOCK_TABLE, ERR_SEL, ERR_NO_VICTIM, ERR_TIMEOUT, ERR_FULL, ERR_INIT = 1, 2,
 EXPORTS = ("nosa_state_sizes", "nosa_workspace_size", "nosa_workspace_init", "nosa_state_init",
            "nosa_append", "nosa_score_blocks", "nosa_select", "nosa_gather", "nosa_decode_attn",
            "nosa_step", "nosa_check_device", "nosa_status_string", "nosa_last_error",
-           "nosa_decode_attn_noalloc", "nosa_uva_read_probe")
+           "nosa_decode_attn_noalloc", "nosa_uva_read_probe", "nosa_plan_ahead", "nosa_prefetch", "nosa_attend")
 
 
 class nosa_config(ctypes.Structure):
@@ -80,6 +80,9 @@ def load(path: Optional[str] = None):
         "nosa_check_device": [stp, vp, ctypes.POINTER(ctypes.c_uint32)],
         "nosa_decode_attn_noalloc": [cfgp, stp, vp, vp, vp, vp],
         "nosa_uva_read_probe": [vp, vp, sz, i32, vp],
+        "nosa_plan_ahead": [cfgp, stp, vp, vp, vp, vp, vp, sz, vp],
+        "nosa_prefetch": [cfgp, stp, vp, sz, vp],
+        "nosa_attend": [cfgp, stp, vp, vp, vp, vp, vp, vp, sz, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -195,6 +198,23 @@ def uva_read_probe(host, dev, nbytes: int, ctas: int = 0, stream=None):
     """Measurement helper: copies nbytes of pinned host memory to device memory by 16-byte UVA
     loads (the gather's access); its time is the PCIe read ceiling of the gather."""
     _check(load().nosa_uva_read_probe(_ptr(host), _ptr(dev), nbytes, ctas, _stream(stream)))
+
+
+def plan_ahead(cfg, st, score_rows, evict, sel, miss_count, ws, ws_bytes, stream=None):
+    """Lookahead call 1: select and plan from score_rows on the cache as it stands."""
+    _check(load().nosa_plan_ahead(ctypes.byref(cfg), ctypes.byref(st), _ptr(score_rows), _ptr(evict),
+                                  _ptr(sel), _ptr(miss_count), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def prefetch(cfg, st, ws, ws_bytes, stream=None):
+    """Lookahead call 2: host -> HBM copies of the planned pages (no-op without host pools)."""
+    _check(load().nosa_prefetch(ctypes.byref(cfg), ctypes.byref(st), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def attend(cfg, st, q, k_new, v_new, sel, out, ws, ws_bytes, stream=None):
+    """Lookahead call 3: append the token, attend over the blocks plan_ahead chose."""
+    _check(load().nosa_attend(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(k_new), _ptr(v_new),
+                              _ptr(sel), _ptr(out), _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def check_device(st, stream=None):

@@ -10,7 +10,8 @@ from typing import Optional
 import torch
 
 from . import (nosa_config, nosa_state, STATE_FIELDS, state_sizes, workspace_size, workspace_init,
-               state_init, append, score_blocks, select, gather, decode_attn, step, check_device)
+               state_init, append, score_blocks, select, gather, decode_attn, step, check_device,
+               plan_ahead, prefetch, attend)
 
 _DTYPE = {"seq_len": torch.int32, "kc": torch.float32, "prev_sel": torch.int32,
           "alive": torch.int32, "last_used": torch.int32, "block_table": torch.int32,
@@ -74,6 +75,16 @@ class NosaCache:
              events=None):
         step(self.cfg, self.state, q, score_rows, k_new, v_new, evict, sel, out, miss_count, self.ws,
              self.ws_bytes, stream, events)
+
+    def plan_ahead(self, score_rows, evict, sel, miss_count, stream=None):
+        plan_ahead(self.cfg, self.state, score_rows, evict, sel, miss_count, self.ws, self.ws_bytes,
+                   stream)
+
+    def prefetch(self, stream=None):
+        prefetch(self.cfg, self.state, self.ws, self.ws_bytes, stream)
+
+    def attend(self, q, k_new, v_new, sel, out, stream=None):
+        attend(self.cfg, self.state, q, k_new, v_new, sel, out, self.ws, self.ws_bytes, stream)
 
     def check(self, stream=None):
         return check_device(self.state, stream)

@@ -286,7 +286,7 @@ nosa_status make_pool_map(CUtensorMap* m, const nosa_config& c, void* pool) {
 // whole PCIe transfer, so spreading each group over more CTAs shortens the last group's tail).
 template <int D, int BS>
 nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& tk, const CUtensorMap& tv,
-                          cudaStream_t s, bool finest) {
+                          cudaStream_t s, bool finest, bool pdl = true) {
   using SH = AttnShape<D, BS>;
   int stages = (110 * 1024) / SH::STAGE;
   stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
@@ -332,15 +332,16 @@ nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& t
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = at;
-  lc.numAttrs = 1;
+  lc.numAttrs = pdl ? 1 : 0;
   NOSA_CUDA(cudaLaunchKernelEx(&lc, k, tk, tv, a));
   return NOSA_OK;
 }
 
 // ready: per-group flags the attention waits on (and clears), or NULL to wait for the
-// previous grid as a whole.
+// previous grid as a whole. pdl: may start while the previous kernel on the stream runs.
 nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16_t* q, const int32_t* sel,
-                        float* out, void* ws, cudaStream_t s, uint32_t* ready = nullptr) {
+                        float* out, void* ws, cudaStream_t s, uint32_t* ready = nullptr,
+                        bool pdl = true) {
   CUtensorMap tk, tv;
   nosa_status r = make_pool_map(&tk, c, st->k_pool);
   if (r != NOSA_OK) return r;
@@ -368,13 +369,13 @@ nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16
   a.sel_flag = ready;
   const bool finest = ready != nullptr && has_host(st);
   if (c.d == 128) {
-    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s, finest);
-    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s, finest);
-    return launch_attn_t<128, 128>(c, a, tk, tv, s, finest);
+    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s, finest, pdl);
+    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s, finest, pdl);
+    return launch_attn_t<128, 128>(c, a, tk, tv, s, finest, pdl);
   }
-  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s, finest);
-  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s, finest);
-  return launch_attn_t<64, 128>(c, a, tk, tv, s, finest);
+  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s, finest, pdl);
+  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s, finest, pdl);
+  return launch_attn_t<64, 128>(c, a, tk, tv, s, finest, pdl);
 }
 
 }  // namespace
@@ -583,6 +584,7 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   a.evict = evict;
   a.sel = sel;
   a.miss_count = miss_count;
+  a.append = 1;
   // Per-group flags chain the kernels group by group: the attention of a group starts as soon
   // as that group's selection is published or, with host pools, as soon as its page copies
   // (which themselves start on the group's published plan) have landed. With events each
@@ -598,6 +600,68 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   if ((r = rec(2)) != NOSA_OK) return r;
   if ((r = launch_attn(c, st, q, sel, out, ws, s, ready)) != NOSA_OK) return r;
   return rec(3);
+}
+
+nosa_status nosa_plan_ahead(const nosa_config* cfg, const nosa_state* st, const uint16_t* score_rows,
+                            const float* evict, int32_t* sel, int32_t* miss_count, void* ws,
+                            size_t ws_bytes, void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
+  NOSA_CHECK(score_rows && evict && sel && miss_count, "plan_ahead buffer is NULL");
+  const void* ptrs[] = {score_rows, evict, sel, miss_count};
+  for (const void* p : ptrs) NOSA_CHECK(aligned16(p), "plan_ahead buffer %p not 16-byte aligned", p);
+  cudaStream_t s = as_stream(stream);
+  const WsLayout w = ws_layout(c);
+  StepArgs a = step_args(c, st);
+  set_ws(a, c, ws);
+  a.rows = score_rows;
+  a.R = c.n_score_rows;
+  a.block_scores = ws_at<float>(ws, w.scores);
+  a.evict = evict;
+  a.sel = sel;
+  a.miss_count = miss_count;
+  a.append = 0;
+  a.sel_flag = ws_at<uint32_t>(ws, w.sel_flag);
+  return launch_score<true>(c, a, s);
+}
+
+nosa_status nosa_prefetch(const nosa_config* cfg, const nosa_state* st, void* ws, size_t ws_bytes,
+                          void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
+  if (!has_host(st)) return NOSA_OK;
+  return launch_copy(c, st, ws, as_stream(stream), true);
+}
+
+nosa_status nosa_attend(const nosa_config* cfg, const nosa_state* st, const uint16_t* q,
+                        const uint16_t* k_new, const uint16_t* v_new, const int32_t* sel, float* out,
+                        void* ws, size_t ws_bytes, void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
+  NOSA_CHECK(q && k_new && v_new && sel && out, "attend buffer is NULL");
+  const void* ptrs[] = {q, k_new, v_new, sel, out};
+  for (const void* p : ptrs) NOSA_CHECK(aligned16(p), "attend buffer %p not 16-byte aligned", p);
+  cudaStream_t s = as_stream(stream);
+  const WsLayout w = ws_layout(c);
+  uint32_t* ready = ws_at<uint32_t>(ws, has_host(st) ? w.copy_flag : w.sel_flag);
+  StepArgs a = step_args(c, st);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.ready = ready;
+  if (c.d == 128) append_kernel<128><<<n_groups(c), 128, 0, s>>>(a);
+  else append_kernel<64><<<n_groups(c), 128, 0, s>>>(a);
+  NOSA_CUDA(cudaGetLastError());
+  // no programmatic early start: the attention reads the length the append just wrote
+  return launch_attn(c, st, q, sel, out, ws, s, ready, false);
 }
 
 nosa_status nosa_check_device(const nosa_state* st, void* stream, uint32_t* err_out) {

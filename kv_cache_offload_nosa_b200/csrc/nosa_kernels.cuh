@@ -51,6 +51,9 @@ struct StepArgs {
   uint32_t* ge_mask;      // [B*Hkv][W] Gamma_e handed from chunk 0 to the last chunk
   uint32_t* sel_flag;     // [B*Hkv * kFlagStride] set (release) once a group's selection is published, or NULL
   uint32_t* err;
+  int append;             // fused score kernel: 1 appends the step's token first, 0 scores the
+                          // cache as it stands (lookahead planning)
+  const uint32_t* ready;  // append_kernel: per-group flags to acquire before writing, or NULL
 };
 
 // Append token pos = len0 of group gi (all threads of the CTA take part).
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
 
   const int len0 = a.seq_len[gi];
   int L = len0;
-  if (FUSED) {
+  if (FUSED && a.append) {
     if (len0 < a.max_blocks * a.bs) L = len0 + 1;
     else if (c == 0 && tid == 0) set_err(a.err, NOSA_ERR_FULL);
   }
@@ -255,6 +258,12 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
 template <int D>
 __global__ void __launch_bounds__(128) append_kernel(StepArgs a) {
   const int gi = blockIdx.x;
+  if (a.ready) {
+    // lookahead: this group's page copies may target the tail block; they land first
+    if (threadIdx.x == 0 && !wait_flag(a.ready + (size_t)gi * kFlagStride, globaltimer() + kWaitLimitNs))
+      set_err(a.err, NOSA_ERR_TIMEOUT);
+    __syncthreads();
+  }
   const int len0 = a.seq_len[gi];
   if (len0 >= a.max_blocks * a.bs) {
     if (threadIdx.x == 0) set_err(a.err, NOSA_ERR_FULL);

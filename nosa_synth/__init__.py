@@ -213,6 +213,16 @@ def configs() -> dict:
     c["bs128_d64"] = NosaConfig("bs128_d64", 2, 16, 2, 64, (3000, 2900), 128, 16, 3, 5, 4,
                                 recipe="sink", cfg_id=54)
     c["g8"] = NosaConfig("g8", 2, 16, 2, 128, (1500, 1537), 64, 32, 5, 6, 3, cfg_id=55)
+    # lookahead (SparDA order: select from the forecast row, then append, then attend)
+    c["lookahead"] = c["offload"].with_(name="lookahead", n_score_rows=1, cfg_id=61)
+    c["lookahead_small"] = c["offload_small"].with_(name="lookahead_small", n_score_rows=1,
+                                                    cfg_id=62)
+    c["lookahead_hbm"] = c["llama_small"].with_(name="lookahead_hbm", n_score_rows=1, cfg_id=63)
+    c["lookahead_ragged"] = c["ragged_offload"].with_(name="lookahead_ragged", n_score_rows=1,
+                                                      cfg_id=64)
+    c["lookahead_tiny"] = c["tiny"].with_(name="lookahead_tiny", n_score_rows=1, cfg_id=65)
+    c["lookahead_dense"] = c["tiny"].with_(name="lookahead_dense", n_score_rows=1, k_q=57,
+                                           cfg_id=66)
     return c
 
 

@@ -202,15 +202,26 @@ class Case:
 
 
 def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = MARGIN,
-             max_retry: int = 64, keep_state: bool = True, lib_path: Optional[str] = None) -> Case:
+             max_retry: int = 64, keep_state: bool = True, lib_path: Optional[str] = None,
+             lookahead: bool = False) -> Case:
     """Generate a config's inputs and run the oracle over its steps.
 
-    Margin enforcement: after each append the query-aware cut of every group is
-    checked; when the fp64 gap between the last selected and the first
+    Margin enforcement: once the step's scores exist the query-aware cut of every
+    group is checked; when the fp64 gap between the last selected and the first
     unselected block score is below `margin`, that group's query (or forecast)
     row is redrawn from the next retry stream. The final inputs are the ones
     recorded, so the GPU and the oracle consume identical arrays.
+
+    lookahead: SparDA's decoupled order (gist.science/de/paper/2606.04511, section 2,
+    "Trainierbare Lookahead Sparse-Selektion"): the blocks a step attends are chosen, and
+    their residency planned, from the forecast row before the step's token is appended;
+    the token is then appended and the query attends over the chosen blocks. Needs a
+    forecast config (one scoring row per group) and a non-empty prefill.
     """
+    if lookahead and cfg.n_score_rows != 1:
+        raise ValueError("lookahead selection scores with the forecast row (n_score_rows == 1)")
+    if lookahead and min(cfg.T) < 1:
+        raise ValueError("lookahead needs a non-empty prefill")
     inp = syn.make_inputs(cfg)
     # the oracle appends in place: inp.pool_k / pool_v rows >= T then hold the decode tokens
     orc = Oracle(cfg, inp.pool_k, inp.pool_v, inp.resident, lib_path, copy=False)
@@ -219,7 +230,8 @@ def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = M
     prev = None
     recs = []
     for t in range(S):
-        orc.append(inp.k_new[t], inp.v_new[t])
+        if not lookahead:
+            orc.append(inp.k_new[t], inp.v_new[t])
         retry = np.zeros((cfg.B, cfg.Hkv), np.int64)
         todo = np.ones(cfg.B * cfg.Hkv, np.uint8)
         scores = np.empty((cfg.B * cfg.Hkv, cfg.max_blocks), np.float64)
@@ -247,6 +259,8 @@ def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = M
         prev = qs
         sel, src, gap = orc.select(scores, inp.evict[t], commit=True)
         miss = orc.residency(sel)
+        if lookahead:
+            orc.append(inp.k_new[t], inp.v_new[t])
         out = orc.attend(q16, sel)
         recs.append(StepRecord(q16, np.ascontiguousarray(rows), fc, scores, sel, src, gap, miss, out,
                                retry, orc.snapshot() if keep_state else {}))

@@ -70,6 +70,12 @@ def run_step(cache, cfg, inputs, rec, t, io: StepIO, mode: str = "fused"):
     ev = dev(inputs.evict[t])
     if mode == "fused":
         cache.step(q, kn, vn, ev, io.sel, io.out, io.miss, score_rows=rows)
+    elif mode == "lookahead":
+        # SparDA order on one stream: select and plan from the forecast row, copy, then
+        # append and attend
+        cache.plan_ahead(rows if rows is not None else q, ev, io.sel, io.miss)
+        cache.prefetch()
+        cache.attend(q, kn, vn, io.sel, io.out)
     else:
         cache.append(kn, vn)
         cache.score_blocks(rows if rows is not None else q, io.scores)

@@ -107,8 +107,10 @@ def _brute_top(keys: dict, m: int):
     return out
 
 
-def check_selection_trace(case):
-    """The pages' invariants plus brute-force top-m of each set on a generated trace."""
+def check_selection_trace(case, lookahead=False):
+    """The pages' invariants plus brute-force top-m of each set on a generated trace.
+
+    lookahead: the step selected before appending its token (length T + t, not T + t + 1)."""
     c = case.cfg
     for gi in range(c.B * c.Hkv):
         b = gi // c.Hkv
@@ -116,7 +118,7 @@ def check_selection_trace(case):
         prev = set(range(n0))
         dropped = set()      # blocks that were in S(t-1) but not kept by Gamma_e(t)
         for t, rec in enumerate(case.steps):
-            Lt = c.T[b] + t + 1
+            Lt = c.T[b] + t + (0 if lookahead else 1)
             N = -(-Lt // c.block)
             S, Ge, Gq = _sets(rec, gi)
             assert S == sorted(set(S)), "S ascending and unique"
@@ -210,14 +212,15 @@ def check_hand_residency(lib_path=None):
         assert orc.last_used[0].tolist() == h["expect_last_used"][t]
 
 
-def check_residency_trace(case):
-    """Invariants of the residency model on a generated offload trace."""
+def check_residency_trace(case, lookahead=False):
+    """Invariants of the residency model on a generated offload trace (lookahead: planned
+    before the step's append, at length T + t)."""
     c = case.cfg
     for t, rec in enumerate(case.steps):
         st = rec.state
         for gi in range(c.B * c.Hkv):
             b = gi // c.Hkv
-            Lt = c.T[b] + t + 1
+            Lt = c.T[b] + t + (0 if lookahead else 1)
             tail = (Lt - 1) // c.block
             S = [int(j) for j in rec.sel[gi] if j >= 0]
             bsl, own = st["block_slot"][gi], st["slot_owner"][gi]
@@ -266,8 +269,35 @@ def check_attention_dense_sdpa(lib_path=None):
             np.testing.assert_allclose(rec.out[b, g * cfg.G:(g + 1) * cfg.G], ref, rtol=1e-11, atol=1e-13)
 
 
-def check_attention_subset(cfg, lib_path=None, steps=None):
-    case = O.run_case(cfg, steps=steps, lib_path=lib_path)
+def check_lookahead_dense_sdpa(lib_path=None):
+    """Lookahead order with every block selected: the step selects the N blocks that exist
+    before its append, then attends after it. So it is plain softmax attention (torch SDPA)
+    over the tokens < L + 1 inside those N blocks: the new token counts only when its block
+    already existed."""
+    cfg = syn.configs()["lookahead_dense"]
+    case = O.run_case(cfg, lib_path=lib_path, lookahead=True)
+    orc = case.oracle
+    for t, rec in enumerate(case.steps):
+        for gi in range(cfg.B * cfg.Hkv):
+            L0 = cfg.T[0] + t                     # length when the step selects
+            N = -(-L0 // cfg.block)
+            assert [int(j) for j in rec.sel[gi] if j >= 0] == list(range(N))
+            n_att = min(L0 + 1, N * cfg.block)   # tokens the step attends
+            K, V = _tokens(orc, gi, L0 + 1)
+            b, g = gi // cfg.Hkv, gi % cfg.Hkv
+            q = torch.from_numpy(syn.bf16_to_f64(rec.q[b, g * cfg.G:(g + 1) * cfg.G]))
+            Kt, Vt = torch.from_numpy(K[:n_att]), torch.from_numpy(V[:n_att])
+            ref = F.scaled_dot_product_attention(q[None, :, None, :], Kt[None, None].expand(1, cfg.G, -1, -1),
+                                                 Vt[None, None].expand(1, cfg.G, -1, -1),
+                                                 scale=cfg.scale)[0, :, 0, :].numpy()
+            np.testing.assert_allclose(rec.out[b, g * cfg.G:(g + 1) * cfg.G], ref, rtol=1e-11, atol=1e-13)
+    return case
+
+
+def check_attention_subset(cfg, lib_path=None, steps=None, lookahead=False):
+    """Output = softmax attention (torch) over the tokens < L_t + 1 of the selected blocks (the
+    length after the step's append, in either order)."""
+    case = O.run_case(cfg, steps=steps, lib_path=lib_path, lookahead=lookahead)
     orc = case.oracle
     for t, rec in enumerate(case.steps):
         for gi in range(cfg.B * cfg.Hkv):

@@ -25,3 +25,13 @@ def test_full_size_parity(name):
     case = O.run_case(CS[name])
     _, (mx, rl2) = H.run_and_compare(case)
     assert mx <= H.ATOL and rl2 <= H.RTOL_L2
+
+
+def test_full_size_lookahead_parity():
+    """The offload workload with a forecast row, in lookahead order, at full size."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gpu_harness as H
+    case = O.run_case(CS["lookahead"], steps=16, lookahead=True)
+    _, (mx, rl2) = H.run_and_compare(case, mode="lookahead")
+    assert mx <= H.ATOL and rl2 <= H.RTOL_L2

@@ -61,6 +61,25 @@ def test_attention_and_selection_trace(name):
         P.check_residency_trace(case)
 
 
+def test_lookahead_dense_equals_sdpa():
+    P.check_lookahead_dense_sdpa()
+
+
+@pytest.mark.parametrize("name", ["lookahead_tiny", "lookahead_ragged", "lookahead_small"])
+def test_lookahead_attention_and_selection_trace(name):
+    case = P.check_attention_subset(CS[name], lookahead=True)
+    P.check_selection_trace(case, lookahead=True)
+    if case.cfg.offload:
+        P.check_residency_trace(case, lookahead=True)
+
+
+def test_lookahead_needs_forecast_rows_and_prefill():
+    with pytest.raises(ValueError):
+        O.run_case(CS["tiny"], steps=1, lookahead=True)
+    with pytest.raises(ValueError):
+        O.run_case(CS["empty"].with_(n_score_rows=1), steps=1, lookahead=True)
+
+
 def test_margin_enforced():
     case = O.run_case(CS["llama_small"])
     for rec in case.steps:
