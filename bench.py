@@ -51,7 +51,8 @@ def workload(name: str, steps: int, batch: int = 0) -> syn.NosaConfig:
 def describe(cfg: syn.NosaConfig) -> str:
     return (f"{cfg.name}: B={cfg.B} Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} T={cfg.T[0]} "
             f"block={cfg.block} sub_block={cfg.sub_block} k={cfg.k} (k_q={cfg.k_q}, k_e={cfg.k_e})"
-            + (f" slots={cfg.slots} offload" if cfg.offload else " all KV in HBM"))
+            + (f" slots={cfg.slots} offload" if cfg.offload else " all KV in HBM")
+            + (f" score_mode={cfg.score_mode}" if cfg.score_mode else ""))
 
 
 def step_bytes(cfg: syn.NosaConfig, L: int, misses: int = 0):
@@ -254,7 +255,7 @@ def run_gpu(args, cfg):
     inp = syn.make_inputs(cfg)
     NG = cfg.B * cfg.Hkv
     cc = nosa.make_config(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.block, cfg.sub_block, cfg.k_q, cfg.k_e,
-                          cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows, scale=cfg.scale)
+                          cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows, scale=cfg.scale, score_mode=cfg.score_mode)
     cache = nosa.NosaCache(cc, offload=cfg.offload)
     pk = torch.from_numpy(inp.pool_k.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)
     pv = torch.from_numpy(inp.pool_v.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)
@@ -499,7 +500,7 @@ def run_lookahead(args, cfg):
     for c in cfgs:
         inp = syn.make_inputs(c)
         cc = nosa.make_config(c.B, c.Hq, c.Hkv, c.d, c.block, c.sub_block, c.k_q, c.k_e, c.max_blocks,
-                              slots=c.n_slots, n_score_rows=c.rows, scale=c.scale)
+                              slots=c.n_slots, n_score_rows=c.rows, scale=c.scale, score_mode=c.score_mode)
         cache = nosa.NosaCache(cc, offload=True)
         cache.pool_view("host_k").copy_(torch.from_numpy(inp.pool_k.reshape(NG, c.max_blocks, c.block, c.d)).view(torch.int16))
         cache.pool_view("host_v").copy_(torch.from_numpy(inp.pool_v.reshape(NG, c.max_blocks, c.block, c.d)).view(torch.int16))

@@ -72,7 +72,18 @@ typedef struct nosa_config {
   int32_t n_score_rows;   /* G: score with the group's query heads; 1: one forecast row */
   int32_t attn_split;     /* selected blocks per attention CTA; 0 = automatic */
   float scale;            /* sigma, the softmax scale (1/sqrt(d) for standard attention) */
+  int32_t score_mode;     /* scoring variant bits, 0 = the NOSA pool (sub-block means, mean of
+                             the rows' raw logits). NOSA_SCORE_WINDOW: units are windows of two
+                             sub-blocks at a stride of one (SparDA's (32, 16) inference window
+                             at sub_block 16, gist.science/de/paper/2606.04511, section 2
+                             "Trainingsstrategie"); NOSA_SCORE_SOFTMAX: per scoring row a softmax
+                             over all units, summed over the rows (needs n_score_rows <= 8).
+                             A block's score is the max over the units starting in it. Variants
+                             run only in nosa_step and nosa_plan_ahead. */
 } nosa_config;
+
+#define NOSA_SCORE_WINDOW 1
+#define NOSA_SCORE_SOFTMAX 2
 
 /*
  * Decode state: caller-allocated buffers, sized by nosa_state_sizes.

@@ -28,10 +28,14 @@ EXPORTS = ("nosa_state_sizes", "nosa_workspace_size", "nosa_workspace_init", "no
            "nosa_decode_attn_noalloc", "nosa_uva_read_probe", "nosa_plan_ahead", "nosa_prefetch", "nosa_attend")
 
 
+NOSA_SCORE_WINDOW, NOSA_SCORE_SOFTMAX = 1, 2
+
+
 class nosa_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "Hq", "Hkv", "d", "block_size", "sub_block", "k_q", "k_e", "max_blocks",
-                 "slots", "n_score_rows", "attn_split")] + [("scale", ctypes.c_float)]
+                 "slots", "n_score_rows", "attn_split")] + [("scale", ctypes.c_float),
+                                                             ("score_mode", ctypes.c_int32)]
 
 
 STATE_FIELDS = ("seq_len", "kc", "prev_sel", "alive", "last_used", "block_table", "slot_owner",
@@ -121,11 +125,11 @@ def _stream(stream) -> Optional[int]:
 
 
 def make_config(B, Hq, Hkv, d, block_size, sub_block, k_q, k_e, max_blocks, slots=None,
-                n_score_rows=None, attn_split=0, scale=None) -> nosa_config:
+                n_score_rows=None, attn_split=0, scale=None, score_mode=0) -> nosa_config:
     G = Hq // Hkv
     return nosa_config(B, Hq, Hkv, d, block_size, sub_block, k_q, k_e, max_blocks,
                        max_blocks if slots is None else slots, G if n_score_rows is None else n_score_rows,
-                       attn_split, (1.0 / d ** 0.5) if scale is None else scale)
+                       attn_split, (1.0 / d ** 0.5) if scale is None else scale, score_mode)
 
 
 def state_sizes(cfg: nosa_config) -> nosa_sizes:

@@ -64,6 +64,10 @@ nosa_status check_cfg(const nosa_config* cp) {
   NOSA_CHECK(c.n_score_rows == G || c.n_score_rows == 1, "n_score_rows = %d must be G or 1",
              c.n_score_rows);
   NOSA_CHECK(c.attn_split >= 0, "attn_split < 0");
+  NOSA_CHECK(c.score_mode >= 0 && c.score_mode <= (NOSA_SCORE_WINDOW | NOSA_SCORE_SOFTMAX),
+             "score_mode = %d: bits NOSA_SCORE_WINDOW | NOSA_SCORE_SOFTMAX only", c.score_mode);
+  NOSA_CHECK(!(c.score_mode & NOSA_SCORE_SOFTMAX) || c.n_score_rows <= kMaxSoftRows,
+             "softmax scoring supports at most %d scoring rows", kMaxSoftRows);
   NOSA_CHECK(c.scale > 0.f, "scale must be > 0");
   const long long groups = (long long)c.B * c.Hkv;
   NOSA_CHECK(groups * c.slots * c.block_size < (1ll << 31), "too many pool rows for TMA coordinates");
@@ -103,7 +107,7 @@ nosa_status check_state(const nosa_config& c, const nosa_state* st) {
 
 struct WsLayout {
   size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, ge_mask, sel_flag, copy_cnt,
-      copy_flag, total;
+      copy_flag, units, total;
   int copy_stride;
 };
 
@@ -125,6 +129,9 @@ WsLayout ws_layout(const nosa_config& c) {
   w.sel_flag = off; off += up256(NG * kFlagStride * 4);
   w.copy_cnt = off; off += up256(NG * 4);
   w.copy_flag = off; off += up256(NG * kFlagStride * 4);
+  // scoring variants: per-sub-block values (rows of logits for softmax, else one mean)
+  const size_t urows = !c.score_mode ? 0 : ((c.score_mode & NOSA_SCORE_SOFTMAX) ? c.n_score_rows : 1);
+  w.units = off; off += up256(NG * urows * (size_t)max_sub(c) * 4);
   w.total = off;
   return w;
 }
@@ -177,11 +184,28 @@ void set_ws(StepArgs& a, const nosa_config& c, void* ws) {
   a.copy_count = ws_at<int32_t>(ws, w.copy_count);
   a.counters = ws_at<uint32_t>(ws, w.cnt_k1);
   a.ge_mask = ws_at<uint32_t>(ws, w.ge_mask);
+  a.mode = c.score_mode;
+  a.units = c.score_mode ? ws_at<float>(ws, w.units) : nullptr;
 }
 
 // ------------------------------------------------------------------ launches
+template <int D, bool FUSED, int VARIANT>
+nosa_status launch_score_t(const nosa_config& c, const StepArgs& a, cudaStream_t s) {
+  dim3 grid((max_sub(c) + kChunkSub - 1) / kChunkSub, n_groups(c));
+  const size_t dsm = FUSED ? sel_smem_bytes(c.max_blocks) : 0;
+  auto k = score_kernel<D, FUSED, VARIANT>;
+  if (dsm > 48 * 1024) NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm));
+  k<<<grid, kScoreThreads, dsm, s>>>(a);
+  NOSA_CUDA(cudaGetLastError());
+  return NOSA_OK;
+}
+
 template <bool FUSED>
 nosa_status launch_score(const nosa_config& c, const StepArgs& a, cudaStream_t s) {
+  if (FUSED && (c.score_mode & NOSA_SCORE_SOFTMAX))
+    return c.d == 128 ? launch_score_t<128, true, 2>(c, a, s) : launch_score_t<64, true, 2>(c, a, s);
+  if (FUSED && c.score_mode)
+    return c.d == 128 ? launch_score_t<128, true, 1>(c, a, s) : launch_score_t<64, true, 1>(c, a, s);
   dim3 grid((max_sub(c) + kChunkSub - 1) / kChunkSub, n_groups(c));
   const size_t dsm = FUSED ? sel_smem_bytes(c.max_blocks) : 0;
   if (c.d == 128) {
@@ -500,6 +524,8 @@ nosa_status nosa_score_blocks(const nosa_config* cfg, const nosa_state* st, cons
   if ((r = check_state(c, st)) != NOSA_OK) return r;
   NOSA_CHECK(rows && block_scores && aligned16(rows) && aligned16(block_scores),
              "score rows / block_scores NULL or misaligned");
+  NOSA_CHECK(c.score_mode == 0, "scoring variants need the whole group's values before any block "
+                                "score: use nosa_step or nosa_plan_ahead");
   StepArgs a = step_args(c, st);
   a.rows = rows;
   a.R = c.n_score_rows;

@@ -54,7 +54,93 @@ struct StepArgs {
   int append;             // fused score kernel: 1 appends the step's token first, 0 scores the
                           // cache as it stands (lookahead planning)
   const uint32_t* ready;  // append_kernel: per-group flags to acquire before writing, or NULL
+  int mode;               // scoring variant bits (1 windows, 2 per-row softmax); 0 = NOSA pool
+  float* units;           // variants: per-sub-block values [B*Hkv][rows][max_sub] (workspace)
 };
+
+constexpr int kMaxSoftRows = 8;  // scoring rows the per-row softmax variant supports
+
+// Block scores of the scoring variants, computed by the last CTA of a group from the
+// per-sub-block values its chunks left in a.units (softmax: sigma q_r . kbar_i per row r;
+// otherwise the mean over the rows). The unit starting at sub-block i is that sub-block or,
+// with windows, the window of sub-blocks i and i+1: its value is the present-token-weighted
+// mean of theirs (the logit of the window's mean key, by linearity). Softmax: per row over
+// all units, then the sum over the rows. Block score = max over the units starting in it.
+// (SparDA, gist.science/de/paper/2606.04511, section 2: the (32, 16) inference window and the
+// per-head softmax scoring its compact indexer removes.)
+template <bool SOFT>
+__device__ void variant_block_scores(const StepArgs& a, int gi, int L, int M, int N, float* red) {
+  const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = nth >> 5;
+  const bool win = (a.mode & 1) != 0;
+  constexpr bool soft = SOFT;
+  const int Ru = soft ? a.R : 1;
+  const int spb = a.bs / a.s;
+  const float* v = a.units + (size_t)gi * Ru * a.max_sub;
+  auto unit = [&](int r, int i) -> float {
+    const float* vr = v + (size_t)r * a.max_sub;
+    const float x0 = __ldcg(vr + i);
+    if (!win || i + 1 >= M) return x0;
+    const int n0 = min(a.s, L - i * a.s), n1 = min(a.s, L - (i + 1) * a.s);
+    return (n0 * x0 + n1 * __ldcg(vr + i + 1)) / (float)(n0 + n1);
+  };
+  float* mx = red;                    // [kMaxSoftRows]
+  float* den = red + kMaxSoftRows;    // [kMaxSoftRows]
+  float* part = red + 2 * kMaxSoftRows;  // [kMaxSoftRows][nw]
+  if constexpr (SOFT) {
+    for (int pass = 0; pass < 2; ++pass) {
+      float acc[kMaxSoftRows];
+#pragma unroll
+      for (int r = 0; r < kMaxSoftRows; ++r) acc[r] = pass == 0 ? -INFINITY : 0.f;
+#pragma unroll 4
+      for (int i = tid; i < M; i += nth) {
+#pragma unroll
+        for (int r = 0; r < kMaxSoftRows; ++r)
+          if (r < Ru) {
+            const float x = unit(r, i);
+            acc[r] = pass == 0 ? fmaxf(acc[r], x) : acc[r] + expf(x - mx[r]);
+          }
+      }
+#pragma unroll
+      for (int r = 0; r < kMaxSoftRows; ++r) {
+        if (r >= Ru) break;
+        float x = acc[r];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+          const float y = __shfl_xor_sync(0xffffffffu, x, o);
+          x = pass == 0 ? fmaxf(x, y) : x + y;
+        }
+        if (lane == 0) part[r * nw + warp] = x;
+      }
+      __syncthreads();
+      if (tid < Ru) {
+        float x = pass == 0 ? -INFINITY : 0.f;
+        for (int w = 0; w < nw; ++w) x = pass == 0 ? fmaxf(x, part[tid * nw + w]) : x + part[tid * nw + w];
+        (pass == 0 ? mx : den)[tid] = x;
+      }
+      __syncthreads();
+    }
+  }
+  for (int j = tid; j < a.max_blocks; j += nth) {
+    float m = -INFINITY;
+    if (j < N) {
+      const int e = min((j + 1) * spb, M);
+      for (int i = j * spb; i < e; ++i) {
+        float p;
+        if constexpr (SOFT) {
+          p = 0.f;
+          for (int r = 0; r < Ru; ++r) p += expf(unit(r, i) - mx[r]) / den[r];
+        } else {
+          p = unit(0, i);
+        }
+        m = fmaxf(m, p);
+      }
+    }
+    a.block_scores[(size_t)gi * a.max_blocks + j] = m;
+  }
+  __threadfence();
+  __syncthreads();
+}
 
 // Append token pos = len0 of group gi (all threads of the CTA take part).
 template <int D>
@@ -94,7 +180,10 @@ __device__ void append_token(const StepArgs& a, int gi, int len0) {
   }
 }
 
-template <int D, bool FUSED>
+// VARIANT: the scoring variants (a.mode != 0; 1: mean of the rows, windows; 2: per-row
+// softmax); the chunks leave per-sub-block values in a.units and the group's last CTA turns
+// them into block scores (fused launches only).
+template <int D, bool FUSED, int VARIANT = 0>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   constexpr int LPS = D / 16;        // lanes per sub-block (16 floats each)
   constexpr int SPW = 32 / LPS;      // sub-blocks per warp pass
@@ -102,6 +191,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   __shared__ float qbar[D];
   __shared__ float su[kChunkSub];
   __shared__ int s_last;
+  __shared__ float vred[VARIANT ? 2 * kMaxSoftRows + kMaxSoftRows * (kScoreThreads / 32) : 1];
   extern __shared__ __align__(16) uint8_t dsm[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -156,8 +246,52 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
     qbar[x] = a.scale * sacc / (float)a.R;
   }
   __syncthreads();
+  constexpr bool soft = VARIANT == 2;
 
-  if (i0 < i1) {
+  if (soft && i0 < i1) {
+    // per-row logits sigma q_r . kbar_i: one sub-block row per LPR lanes (one float4 each),
+    // the group's rows in registers; warp-uniform trip count so the shuffles see full warps
+    constexpr int LPR = D / 4, RPW = 32 / LPR, WROWS = RPW * (kScoreThreads / 32);
+    const int sub2 = lane / LPR, p2 = lane % LPR;
+    float4 qv[kMaxSoftRows];
+#pragma unroll
+    for (int r = 0; r < kMaxSoftRows; ++r) {
+      qv[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < a.R) {
+        const uint16_t* qr = a.rows + ((size_t)gi * a.R + r) * D + 4 * p2;
+        qv[r] = make_float4(a.scale * bf16_bits_to_f32(qr[0]), a.scale * bf16_bits_to_f32(qr[1]),
+                            a.scale * bf16_bits_to_f32(qr[2]), a.scale * bf16_bits_to_f32(qr[3]));
+      }
+    }
+    constexpr int RF = 4;  // rows in flight per warp
+    for (int b0 = i0 + warp * RPW; b0 < i1; b0 += RF * WROWS) {
+      float4 x[RF];
+#pragma unroll
+      for (int f = 0; f < RF; ++f) {
+        const int i = b0 + f * WROWS + sub2;
+        x[f] = (i < i1) ? __ldcs(kcg + (size_t)i * (D / 4) + p2) : make_float4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int r = 0; r < kMaxSoftRows; ++r) {
+        if (r >= a.R) break;
+        float z[RF];
+#pragma unroll
+        for (int f = 0; f < RF; ++f)
+          z[f] = qv[r].x * x[f].x + qv[r].y * x[f].y + qv[r].z * x[f].z + qv[r].w * x[f].w;
+#pragma unroll
+        for (int o = LPR / 2; o >= 1; o >>= 1)
+#pragma unroll
+          for (int f = 0; f < RF; ++f) z[f] += __shfl_xor_sync(0xffffffffu, z[f], o);
+        float* ur = a.units + ((size_t)gi * a.R + r) * a.max_sub;
+#pragma unroll
+        for (int f = 0; f < RF; ++f) {
+          const int i = b0 + f * WROWS + sub2;
+          if (p2 == 0 && i < i1) ur[i] = z[f];
+        }
+      }
+    }
+  }
+  if (!soft && i0 < i1) {
     float qr[16];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
@@ -198,8 +332,12 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
     }
   }
   __syncthreads();
+  if (VARIANT && !soft) {
+    // the mean-of-rows values of the chunk's sub-blocks, for the group's last CTA
+    for (int i = i0 + tid; i < i1; i += kScoreThreads) a.units[(size_t)gi * a.max_sub + i] = su[i - i0];
+  }
   // block max over present sub-blocks; -inf for blocks not yet created
-  {
+  if (!VARIANT) {
     const int j = i0 / spb + tid;
     if (tid < kChunkSub / spb && j < a.max_blocks) {
       float m = -INFINITY;
@@ -219,6 +357,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  if (VARIANT) variant_block_scores<VARIANT == 2>(a, gi, L, M, N, vred);
   const SelSmem S = sel_smem_carve(dsm, a.max_blocks);
   const int k = a.k_q + a.k_e;
   select_query(S, a.block_scores + (size_t)gi * a.max_blocks, a.ge_mask + (size_t)gi * Wmax,

@@ -127,6 +127,7 @@ class NosaConfig:
     seed: int = 0
     n_planted: int = 8
     plant_shift: float = 1.5
+    score_mode: int = 0        # scoring variant bits: 1 overlapping windows, 2 per-row softmax
 
     @property
     def G(self) -> int:
@@ -223,6 +224,17 @@ def configs() -> dict:
     c["lookahead_tiny"] = c["tiny"].with_(name="lookahead_tiny", n_score_rows=1, cfg_id=65)
     c["lookahead_dense"] = c["tiny"].with_(name="lookahead_dense", n_score_rows=1, k_q=57,
                                            cfg_id=66)
+    # scoring variants: overlapping (2s, s) windows, per-row softmax then sum, both
+    for m, tag in ((1, "window"), (2, "softmax"), (3, "window_softmax")):
+        c[f"tiny_{tag}"] = c["tiny"].with_(name=f"tiny_{tag}", score_mode=m, cfg_id=70 + m)
+        c[f"ragged_{tag}"] = c["ragged_offload"].with_(name=f"ragged_{tag}", score_mode=m,
+                                                       cfg_id=73 + m)
+        c[f"llama_small_{tag}"] = c["llama_small"].with_(name=f"llama_small_{tag}", score_mode=m,
+                                                         cfg_id=76 + m)
+    c["llama_window"] = c["llama"].with_(name="llama_window", score_mode=1, cfg_id=81)
+    c["llama_softmax"] = c["llama"].with_(name="llama_softmax", score_mode=2, cfg_id=82)
+    c["forecast_softmax"] = c["tiny_forecast"].with_(name="forecast_softmax", score_mode=2,
+                                                     cfg_id=83)
     return c
 
 

@@ -48,7 +48,7 @@ def build(force: bool = False) -> str:
 class OrcCfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "Hq", "Hkv", "d", "bs", "s", "k_q", "k_e", "n_rows", "max_blocks", "slots",
-                 "offload")] + [("scale", ctypes.c_double)]
+                 "offload", "score_mode")] + [("scale", ctypes.c_double)]
 
 
 class OrcState(ctypes.Structure):
@@ -109,7 +109,7 @@ class Oracle:
         c = cfg
         NG, nb = c.B * c.Hkv, c.max_blocks
         self.c = OrcCfg(c.B, c.Hq, c.Hkv, c.d, c.block, c.sub_block, c.k_q, c.k_e, c.rows, nb,
-                        c.n_slots, int(c.offload), c.scale)
+                        c.n_slots, int(c.offload), int(c.score_mode), c.scale)
         # copy=False: the oracle appends into the caller's arrays (rows >= T change)
         self.K = np.ascontiguousarray(pool_k)
         self.V = np.ascontiguousarray(pool_v)
@@ -201,6 +201,21 @@ class Case:
     steps: List[StepRecord]
 
 
+def _log_gap(scores, sel, src, gap):
+    """The query-aware cut's margin in log units: softmax scores are probabilities of order
+    1/M, so their absolute gaps say nothing about how safely fp32 ranks them; the ratio of
+    the last selected to the first unselected score does."""
+    out = np.array(gap, dtype=np.float64, copy=True)
+    for gi in range(scores.shape[0]):
+        if not np.isfinite(out[gi]):
+            continue
+        q = [int(j) for j, w in zip(sel[gi], src[gi]) if j >= 0 and w == 2]
+        lo = min(scores[gi][j] for j in q)
+        nxt = lo - out[gi]
+        out[gi] = np.log(lo) - np.log(nxt) if nxt > 0 else np.inf
+    return out
+
+
 def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = MARGIN,
              max_retry: int = 64, keep_state: bool = True, lib_path: Optional[str] = None,
              lookahead: bool = False) -> Case:
@@ -247,7 +262,9 @@ def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = M
             else:
                 rows = q16.reshape(cfg.B, cfg.Hkv, G, cfg.d)
             orc.block_scores(rows, out=scores, gmask=todo)
-            _, _, gap = orc.select(scores, inp.evict[t], commit=False, gmask=todo, out=prev_out)
+            sel_t, src_t, gap = orc.select(scores, inp.evict[t], commit=False, gmask=todo, out=prev_out)
+            if cfg.score_mode & 2:
+                gap = _log_gap(scores, sel_t, src_t, gap)
             bad = (gap < margin) & (todo != 0)
             if not bad.any():
                 break

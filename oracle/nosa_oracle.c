@@ -59,6 +59,7 @@ typedef struct {
   int32_t max_blocks;     /* blocks per group the caches can hold */
   int32_t slots;          /* HBM slots per group (offload model) */
   int32_t offload;        /* 1: model HBM residency */
+  int32_t score_mode;     /* scoring variant bits, see orc_block_scores (0: the NOSA pool) */
   double scale;           /* sigma = 1/sqrt(d) */
 } orc_cfg;
 
@@ -186,32 +187,76 @@ void orc_append(const orc_cfg* c, orc_state* st, const uint16_t* k_new, const ui
 }
 
 /* Block scores of the two-stage pool; blocks at or beyond N get -INFINITY.
- * gmask (NULL = all) restricts the call to the groups with gmask[gi] != 0. */
+ * gmask (NULL = all) restricts the call to the groups with gmask[gi] != 0.
+ *
+ * Scoring variants (score_mode bits; 0 is the pool described at the top):
+ *   1  windows: the unit that starts at sub-block i pools the tokens [i*s, i*s + 2s) (its
+ *      present ones) instead of [i*s, (i+1)*s): SparDA's inference window of kernel 32 and
+ *      stride 16 at s = 16 (gist.science/de/paper/2606.04511, section 2,
+ *      "Trainingsstrategie"). Its mean key is the count-weighted mean of the sub-block means
+ *      of sub-blocks i and i+1, which is the mean over the window's tokens.
+ *   2  softmax: for each scoring row r a softmax over all the group's units of
+ *      sigma * (q_r . mean key), summed over the rows (the per-head scoring loop with
+ *      softmax that SparDA's compact indexer removes, section 2 "Kompakter
+ *      Forecast-Indexer"), instead of the mean of the raw logits.
+ * Block score: the max over the units that start inside the block. */
 void orc_block_scores(const orc_cfg* c, const orc_state* st, const uint16_t* rows, double* scores,
                       const uint8_t* gmask) {
   const int NG = n_groups(c), nb = c->max_blocks, MS = max_sub(c), spb = c->bs / c->s;
   const int R = c->n_rows;
+  const int win = (c->score_mode & 1) != 0, soft = (c->score_mode & 2) != 0;
 #pragma omp parallel for schedule(dynamic)
   for (int gi = 0; gi < NG; ++gi) {
     if (gmask && !gmask[gi]) continue;
     const int L = st->len[gi];
-    const int N = cdiv(L, c->bs), M = cdiv(L, c->s);
+    const int M = cdiv(L, c->s);
     double* out = scores + (size_t)gi * nb;
     for (int j = 0; j < nb; ++j) out[j] = -INFINITY;
+    if (M == 0) continue;
+    double* z = (double*)malloc(sizeof(double) * (size_t)R * M);   /* logits [r][i] */
+    double* kb = (double*)malloc(sizeof(double) * c->d);
     for (int i = 0; i < M; ++i) {
-      const double* kb = st->kbar + ((size_t)gi * MS + i) * c->d;
-      double u = 0.0;
+      const double* k0 = st->kbar + ((size_t)gi * MS + i) * c->d;
+      const int n0 = (L - i * c->s < c->s) ? L - i * c->s : c->s;
+      int n1 = 0;
+      if (win && i + 1 < M) n1 = (L - (i + 1) * c->s < c->s) ? L - (i + 1) * c->s : c->s;
+      for (int x = 0; x < c->d; ++x) kb[x] = k0[x];
+      if (n1 > 0) {
+        const double* k1 = st->kbar + ((size_t)gi * MS + i + 1) * c->d;
+        for (int x = 0; x < c->d; ++x) kb[x] = (n0 * k0[x] + n1 * k1[x]) / (double)(n0 + n1);
+      }
       for (int r = 0; r < R; ++r) {
         const uint16_t* q = rows + ((size_t)gi * R + r) * c->d;
         double dot = 0.0;
         for (int x = 0; x < c->d; ++x) dot += bf(q[x]) * kb[x];
-        u += c->scale * dot;
+        z[(size_t)r * M + i] = c->scale * dot;
       }
-      u /= (double)R;
+    }
+    double* mx = (double*)malloc(sizeof(double) * 2 * R);  /* per row: max, sum of exp */
+    double* den = mx + R;
+    if (soft) {
+      for (int r = 0; r < R; ++r) {
+        const double* zr = z + (size_t)r * M;
+        mx[r] = -INFINITY;
+        den[r] = 0.0;
+        for (int i = 0; i < M; ++i) if (zr[i] > mx[r]) mx[r] = zr[i];
+        for (int i = 0; i < M; ++i) den[r] += exp(zr[i] - mx[r]);
+      }
+    }
+    for (int i = 0; i < M; ++i) {
+      double u = 0.0;
+      if (soft) {
+        for (int r = 0; r < R; ++r) u += exp(z[(size_t)r * M + i] - mx[r]) / den[r];
+      } else {
+        for (int r = 0; r < R; ++r) u += z[(size_t)r * M + i];
+        u /= (double)R;
+      }
       const int j = i / spb;
       if (u > out[j]) out[j] = u;
     }
-    (void)N;
+    free(mx);
+    free(kb);
+    free(z);
   }
 }
 

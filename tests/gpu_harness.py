@@ -18,7 +18,7 @@ RTOL_L2 = 1e-3   # relative L2 error of the attention output vs fp64
 def c_config(cfg: syn.NosaConfig, attn_split: int = 0) -> nosa.nosa_config:
     return nosa.make_config(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.block, cfg.sub_block, cfg.k_q, cfg.k_e,
                             cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows,
-                            attn_split=attn_split, scale=cfg.scale)
+                            attn_split=attn_split, scale=cfg.scale, score_mode=cfg.score_mode)
 
 
 def dev(a: np.ndarray) -> torch.Tensor:

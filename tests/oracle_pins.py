@@ -309,6 +309,39 @@ def check_attention_subset(cfg, lib_path=None, steps=None, lookahead=False):
     return case
 
 
+def check_score_variants(cfg, lib_path=None, steps=2):
+    """Scoring variants against torch pooling of token-level logits: units are means of the
+    logits over [i*s, i*s + w) (w = 2s for windows, s otherwise; avg_pool1d of the logits
+    and of a ones mask over a zero-padded row, so partial units divide by their present
+    tokens), softmax over the units of each row then summed over rows (or the mean over
+    rows), and the block score is max_pool1d over each block's units."""
+    case = O.run_case(cfg, steps=steps, lib_path=lib_path)
+    orc, c = case.oracle, case.cfg
+    s, spb = c.sub_block, c.block // c.sub_block
+    w = 2 * s if c.score_mode & 1 else s
+    for t, rec in enumerate(case.steps):
+        for gi in range(c.B * c.Hkv):
+            b, g = gi // c.Hkv, gi % c.Hkv
+            Lt = c.T[b] + t + 1
+            M, N = -(-Lt // s), -(-Lt // c.block)
+            K, _ = _tokens(orc, gi, Lt)
+            rows = syn.bf16_to_f64(rec.rows[b, g] if c.n_score_rows == 1 else rec.q[b, g * c.G:(g + 1) * c.G])
+            rows = rows.reshape(-1, c.d)
+            z = torch.from_numpy(c.scale * rows @ K.T)[None]               # [1, R, Lt]
+            pad = M * s + (w - s) - Lt
+            ones = torch.ones_like(z)
+            sums = F.avg_pool1d(F.pad(z, (0, pad)), w, s) * w
+            cnts = F.avg_pool1d(F.pad(ones, (0, pad)), w, s) * w
+            unit = (sums / cnts)[0]                                         # [R, M]
+            assert unit.shape[1] == M
+            u = torch.softmax(unit, dim=1).sum(0) if c.score_mode & 2 else unit.mean(0)
+            blk = F.max_pool1d(u[None, None], spb, spb, ceil_mode=True)[0, 0].numpy()
+            assert blk.shape[0] == N
+            np.testing.assert_allclose(rec.scores[gi][:N], blk, rtol=1e-10, atol=1e-14)
+            assert np.all(np.isneginf(rec.scores[gi][N:]))
+    return case
+
+
 def run_all(lib_path=None):
     cs = syn.configs()
     check_topm_bruteforce(lib_path, trials=120)
@@ -316,6 +349,8 @@ def run_all(lib_path=None):
     check_hand_residency(lib_path)
     check_static_closed_form(lib_path)
     check_attention_dense_sdpa(lib_path)
+    for name in ("tiny_window", "ragged_window_softmax", "forecast_softmax", "ragged_window"):
+        check_score_variants(cs[name], lib_path)
     for name in ("ragged", "tiny_forecast", "bs128_d64"):
         check_pooling_library(cs[name], lib_path, steps=2)
     for name in ("ragged", "ragged_offload", "g8"):

@@ -44,7 +44,8 @@ def cfg(**kw):
 @pytest.mark.parametrize("bad", [dict(d=96), dict(block_size=48), dict(sub_block=24),
                                  dict(Hq=12, Hkv=4, ), dict(Hq=7), dict(k_q=0, k_e=0),
                                  dict(k_q=30, k_e=20), dict(max_blocks=9000), dict(slots=0),
-                                 dict(n_score_rows=2), dict(scale=0.0), dict(sub_block=128)])
+                                 dict(n_score_rows=2), dict(scale=0.0), dict(sub_block=128),
+                                 dict(score_mode=4), dict(score_mode=-1)])
 def test_bad_config_is_rejected_on_host(lib, bad):
     c = cfg(**bad)
     n = ctypes.c_size_t()
@@ -62,6 +63,18 @@ def test_sizes_follow_the_documented_layout(lib):
     assert s.k_pool == NG * nb_ * bs * d * 2
     assert s.host_k == NG * nb_ * bs * d * 2
     assert nosa.workspace_size(c) > 0
+
+
+def test_score_variants_reserve_their_values(lib):
+    """Variants keep per-sub-block values in the workspace: one per sub-block for windows of
+    the mean, one per scoring row and sub-block for softmax."""
+    base = nosa.workspace_size(cfg())
+    NG, max_sub = 4, 40 * 4
+    win = nosa.workspace_size(cfg(score_mode=nosa.NOSA_SCORE_WINDOW))
+    soft = nosa.workspace_size(cfg(score_mode=nosa.NOSA_SCORE_SOFTMAX))
+    assert win - base >= NG * max_sub * 4
+    assert soft - base >= NG * 4 * max_sub * 4      # G = 4 rows
+    assert nosa.workspace_size(cfg(score_mode=3, n_score_rows=1)) - base >= NG * max_sub * 4
 
 
 def test_status_strings(lib):

@@ -37,6 +37,12 @@ MUTANTS = {
         ("need[tail] = 1;", "need[tail] = 0;"),
     "free slots ignored":
         ("if (own[z] < 0) zl[nz++] = z;", "if (own[z] < -1) zl[nz++] = z;"),
+    "window pools one sub-block":
+        ("if (win && i + 1 < M) n1 =", "if (0 && win && i + 1 < M) n1 ="),
+    "window weights its sub-blocks equally":
+        ("kb[x] = (n0 * k0[x] + n1 * k1[x]) / (double)(n0 + n1);", "kb[x] = 0.5 * (k0[x] + k1[x]);"),
+    "softmax without its normalizer":
+        ("u += exp(z[(size_t)r * M + i] - mx[r]) / den[r];", "u += exp(z[(size_t)r * M + i] - mx[r]);"),
 }
 
 

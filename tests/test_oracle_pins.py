@@ -61,6 +61,13 @@ def test_attention_and_selection_trace(name):
         P.check_residency_trace(case)
 
 
+@pytest.mark.parametrize("name", ["tiny_window", "tiny_softmax", "tiny_window_softmax", "ragged_window",
+                                  "ragged_softmax", "ragged_window_softmax", "forecast_softmax",
+                                  "llama_small_window_softmax"])
+def test_score_variants_equal_torch_pooling(name):
+    P.check_score_variants(CS[name])
+
+
 def test_lookahead_dense_equals_sdpa():
     P.check_lookahead_dense_sdpa()
 
