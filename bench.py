@@ -53,10 +53,11 @@ def describe(cfg: syn.NosaConfig) -> str:
     return (f"{cfg.name}: B={cfg.B} Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} T={cfg.T[0]} "
             f"block={cfg.block} sub_block={cfg.sub_block} k={cfg.k} (k_q={cfg.k_q}, k_e={cfg.k_e})"
             + (f" slots={cfg.slots} offload" if cfg.offload else " all KV in HBM")
-            + (f" score_mode={cfg.score_mode}" if cfg.score_mode else ""))
+            + (f" score_mode={cfg.score_mode}" if cfg.score_mode else "")
+            + (f" stop_tau={cfg.stop_tau}" if cfg.stop_tau else ""))
 
 
-def step_bytes(cfg: syn.NosaConfig, L: int, misses: int = 0):
+def step_bytes(cfg: syn.NosaConfig, L: int, misses: int = 0, visited: float = None):
     """Algorithmic bytes of one step at context length L (after the append), per step.
 
     `misses`: pages (K and V each) the step copied from host memory; each is read over PCIe
@@ -66,6 +67,8 @@ def step_bytes(cfg: syn.NosaConfig, L: int, misses: int = 0):
     N = -(-L // bs)
     M = -(-L // cfg.sub_block)
     nsel = min(cfg.k, N)
+    if visited is not None:  # early stop: pages actually streamed per group
+        nsel = min(nsel, visited)
     tail_tokens = L - (N - 1) * bs
     # K and V of the selected blocks; the tail block (always among them once k >= N) at its
     # present tokens only when it is selected -- counted as full pages otherwise
@@ -256,7 +259,8 @@ def run_gpu(args, cfg):
     inp = syn.make_inputs(cfg)
     NG = cfg.B * cfg.Hkv
     cc = nosa.make_config(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.block, cfg.sub_block, cfg.k_q, cfg.k_e,
-                          cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows, scale=cfg.scale, score_mode=cfg.score_mode)
+                          cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows, scale=cfg.scale, score_mode=cfg.score_mode,
+                          stop_tau=cfg.stop_tau)
     cache = nosa.NosaCache(cc, offload=cfg.offload)
     pk = torch.from_numpy(inp.pool_k.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)
     pv = torch.from_numpy(inp.pool_v.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)
@@ -435,6 +439,14 @@ def run_gpu(args, cfg):
         raise RuntimeError(f"device fault in timed steps: rc={rc} err={err}")
 
     misses = miss_all.sum(dim=1).cpu().numpy()  # K (and V) pages copied per step
+    visited = None
+    if cfg.stop_tau > 0:
+        # early stop: a group streams the blocks its most persistent head visits (counts of
+        # the last step, taken as representative of the timed ones)
+        used = torch.empty(cfg.B * cfg.Hq, dtype=torch.int32, device="cuda")
+        cache.stop_counts(used)
+        per_group = used.view(cfg.B * cfg.Hkv, cfg.G).max(dim=1).values.float()
+        visited = float(per_group.mean().item())
     pcie_peak = pcie_ceiling(nosa, torch) if cfg.offload else None
     # max over ranks
     tot_ms, e2e_ms = D.max_over_ranks([tot_ms, e2e_ms], device="cuda")
@@ -445,10 +457,10 @@ def run_gpu(args, cfg):
     q_per_step = cfg.B * cfg.Hq * world
     value = q_per_step * args.steps / (tot_ms / 1e3)
     hbm_peak, peak_kind = peaks()
-    step_b = [step_bytes(cfg, L, int(misses[ti]))[0] for L, ti in Ls]
+    step_b = [step_bytes(cfg, L, int(misses[ti]), visited)[0] for L, ti in Ls]
     pcie_b = [step_bytes(cfg, L, int(misses[ti]))[3] for L, ti in Ls]
     hbm_gbs = sum(step_b) / (tot_ms / 1e3) / 1e9
-    attn_b = [step_bytes(cfg, L)[1] for L, _ in prof_L]
+    attn_b = [step_bytes(cfg, L, 0, visited)[1] for L, _ in prof_L]
     attn_ms = float(np.mean(k_attn))
     achieved = float(np.mean(attn_b)) / (attn_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -500,6 +512,9 @@ def run_gpu(args, cfg):
     }
     if pcie is not None:
         line["pcie"] = pcie
+    if visited is not None:
+        line["early_stop"] = {"tau": cfg.stop_tau, "blocks_streamed_per_group": visited, "k": cfg.k,
+                              "kernel": "attn_stop_kernel (one CTA per group)"}
     if not args.no_cpu_baseline:
         cb, _ = oracle_sample(workload(args.workload, 4), 3, budget_s=args.cpu_budget)
         line["cpu_baseline"] = cb

@@ -80,6 +80,12 @@ typedef struct nosa_config {
                              over all units, summed over the rows (needs n_score_rows <= 8).
                              A block's score is the max over the units starting in it. Variants
                              run only in nosa_step and nosa_plan_ahead. */
+  float stop_tau;         /* > 0: S2O's monotone-gain early stop (gist.science/it/paper/2602.22575,
+                             "Regola di Arresto Anticipato") in nosa_step: each query head visits
+                             the selected blocks in decreasing block score (ties: lower index) and
+                             stops after the first block whose gain in softmax mass is below
+                             stop_tau times the mass accumulated so far, that block included.
+                             0: attend every selected block. Needs k <= 1024. */
 } nosa_config;
 
 #define NOSA_SCORE_WINDOW 1
@@ -268,6 +274,14 @@ nosa_status nosa_decode_attn_noalloc(const nosa_config* cfg, const nosa_state* s
  * otherwise, or when host is not pinned, device-mapped host memory. Asynchronous on stream.
  */
 nosa_status nosa_uva_read_probe(const void* host, void* dev, size_t bytes, int ctas, void* stream);
+
+/*
+ * Early stop bookkeeping: copies, for the last nosa_step run with stop_tau > 0 on this
+ * workspace, the number of blocks each query head visited into used (device, [B][Hq] int32,
+ * 16-byte aligned). Asynchronous on stream.
+ */
+nosa_status nosa_stop_counts(const nosa_config* cfg, const void* workspace, size_t ws_bytes,
+                             int32_t* used, void* stream);
 
 /* Synchronises the stream, reads state->err into *err_out (may be NULL):
  * NOSA_OK, NOSA_EDEVICE or NOSA_ETIMEOUT. */

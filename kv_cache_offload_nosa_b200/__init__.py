@@ -25,7 +25,7 @@ ERR_BLOCK_TABLE, ERR_SEL, ERR_NO_VICTIM, ERR_TIMEOUT, ERR_FULL, ERR_INIT = 1, 2,
 EXPORTS = ("nosa_state_sizes", "nosa_workspace_size", "nosa_workspace_init", "nosa_state_init",
            "nosa_append", "nosa_score_blocks", "nosa_select", "nosa_gather", "nosa_decode_attn",
            "nosa_step", "nosa_check_device", "nosa_status_string", "nosa_last_error",
-           "nosa_decode_attn_noalloc", "nosa_uva_read_probe", "nosa_plan_ahead", "nosa_prefetch", "nosa_attend")
+           "nosa_decode_attn_noalloc", "nosa_uva_read_probe", "nosa_plan_ahead", "nosa_prefetch", "nosa_attend", "nosa_stop_counts")
 
 
 NOSA_SCORE_WINDOW, NOSA_SCORE_SOFTMAX = 1, 2
@@ -35,7 +35,8 @@ class nosa_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "Hq", "Hkv", "d", "block_size", "sub_block", "k_q", "k_e", "max_blocks",
                  "slots", "n_score_rows", "attn_split")] + [("scale", ctypes.c_float),
-                                                             ("score_mode", ctypes.c_int32)]
+                                                             ("score_mode", ctypes.c_int32),
+                                                             ("stop_tau", ctypes.c_float)]
 
 
 STATE_FIELDS = ("seq_len", "kc", "prev_sel", "alive", "last_used", "block_table", "slot_owner",
@@ -86,6 +87,7 @@ def load(path: Optional[str] = None):
         "nosa_uva_read_probe": [vp, vp, sz, i32, vp],
         "nosa_plan_ahead": [cfgp, stp, vp, vp, vp, vp, vp, sz, vp],
         "nosa_prefetch": [cfgp, stp, vp, sz, vp],
+        "nosa_stop_counts": [cfgp, vp, sz, vp, vp],
         "nosa_attend": [cfgp, stp, vp, vp, vp, vp, vp, vp, sz, vp],
     }
     for name, args in sig.items():
@@ -125,11 +127,11 @@ def _stream(stream) -> Optional[int]:
 
 
 def make_config(B, Hq, Hkv, d, block_size, sub_block, k_q, k_e, max_blocks, slots=None,
-                n_score_rows=None, attn_split=0, scale=None, score_mode=0) -> nosa_config:
+                n_score_rows=None, attn_split=0, scale=None, score_mode=0, stop_tau=0.0) -> nosa_config:
     G = Hq // Hkv
     return nosa_config(B, Hq, Hkv, d, block_size, sub_block, k_q, k_e, max_blocks,
                        max_blocks if slots is None else slots, G if n_score_rows is None else n_score_rows,
-                       attn_split, (1.0 / d ** 0.5) if scale is None else scale, score_mode)
+                       attn_split, (1.0 / d ** 0.5) if scale is None else scale, score_mode, stop_tau)
 
 
 def state_sizes(cfg: nosa_config) -> nosa_sizes:
@@ -219,6 +221,11 @@ def attend(cfg, st, q, k_new, v_new, sel, out, ws, ws_bytes, stream=None):
     """Lookahead call 3: append the token, attend over the blocks plan_ahead chose."""
     _check(load().nosa_attend(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(k_new), _ptr(v_new),
                               _ptr(sel), _ptr(out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def stop_counts(cfg, ws, ws_bytes, used, stream=None):
+    """Blocks each query head visited in the last early-stop step ([B*Hq] int32, device)."""
+    _check(load().nosa_stop_counts(ctypes.byref(cfg), _ptr(ws), ws_bytes, _ptr(used), _stream(stream)))
 
 
 def check_device(st, stream=None):

@@ -11,7 +11,7 @@ import torch
 
 from . import (nosa_config, nosa_state, STATE_FIELDS, state_sizes, workspace_size, workspace_init,
                state_init, append, score_blocks, select, gather, decode_attn, step, check_device,
-               plan_ahead, prefetch, attend)
+               plan_ahead, prefetch, attend, stop_counts)
 
 _DTYPE = {"seq_len": torch.int32, "kc": torch.float32, "prev_sel": torch.int32,
           "alive": torch.int32, "last_used": torch.int32, "block_table": torch.int32,
@@ -85,6 +85,9 @@ class NosaCache:
 
     def attend(self, q, k_new, v_new, sel, out, stream=None):
         attend(self.cfg, self.state, q, k_new, v_new, sel, out, self.ws, self.ws_bytes, stream)
+
+    def stop_counts(self, used, stream=None):
+        stop_counts(self.cfg, self.ws, self.ws_bytes, used, stream)
 
     def check(self, stream=None):
         return check_device(self.state, stream)

@@ -6,6 +6,7 @@
 
 #include "nosa.h"
 #include "nosa_attn.cuh"
+#include "nosa_attn_stop.cuh"
 #include "nosa_common.cuh"
 #include "nosa_kernels.cuh"
 #include "nosa_select.cuh"
@@ -68,6 +69,8 @@ nosa_status check_cfg(const nosa_config* cp) {
              "score_mode = %d: bits NOSA_SCORE_WINDOW | NOSA_SCORE_SOFTMAX only", c.score_mode);
   NOSA_CHECK(!(c.score_mode & NOSA_SCORE_SOFTMAX) || c.n_score_rows <= kMaxSoftRows,
              "softmax scoring supports at most %d scoring rows", kMaxSoftRows);
+  NOSA_CHECK(c.stop_tau >= 0.f && c.stop_tau < 1e30f, "stop_tau must be >= 0 and finite");
+  NOSA_CHECK(!(c.stop_tau > 0.f) || kk(c) <= kStopMaxK, "early stop supports k <= %d", kStopMaxK);
   NOSA_CHECK(c.scale > 0.f, "scale must be > 0");
   const long long groups = (long long)c.B * c.Hkv;
   NOSA_CHECK(groups * c.slots * c.block_size < (1ll << 31), "too many pool rows for TMA coordinates");
@@ -107,7 +110,7 @@ nosa_status check_state(const nosa_config& c, const nosa_state* st) {
 
 struct WsLayout {
   size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, ge_mask, sel_flag, copy_cnt,
-      copy_flag, units, total;
+      copy_flag, units, used, total;
   int copy_stride;
 };
 
@@ -132,6 +135,7 @@ WsLayout ws_layout(const nosa_config& c) {
   // scoring variants: per-sub-block values (rows of logits for softmax, else one mean)
   const size_t urows = !c.score_mode ? 0 : ((c.score_mode & NOSA_SCORE_SOFTMAX) ? c.n_score_rows : 1);
   w.units = off; off += up256(NG * urows * (size_t)max_sub(c) * 4);
+  w.used = off; off += up256((size_t)c.B * c.Hq * 4);
   w.total = off;
   return w;
 }
@@ -361,6 +365,33 @@ nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& t
   return NOSA_OK;
 }
 
+template <int D, int BS>
+nosa_status launch_attn_stop_t(const nosa_config& c, AttnArgs a, StopArgs x, const CUtensorMap& tk,
+                               const CUtensorMap& tv, cudaStream_t s, bool pdl) {
+  using SH = AttnShape<D, BS>;
+  using SS = StopShape<D, BS>;
+  // one CTA per group, one per SM: spend the shared memory on stages
+  const int G = c.Hq / c.Hkv;
+  int stages = (int)((200 * 1024 - SS::extra_bytes(G)) / SH::STAGE);
+  stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
+  const size_t smem = SS::smem_bytes(stages, G);
+  auto k = attn_stop_kernel<D, BS>;
+  NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  a.stages = stages;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(n_groups(c));
+  lc.blockDim = dim3(SH::THREADS);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = pdl ? 1 : 0;
+  NOSA_CUDA(cudaLaunchKernelEx(&lc, k, tk, tv, a, x));
+  return NOSA_OK;
+}
+
 // ready: per-group flags the attention waits on (and clears), or NULL to wait for the
 // previous grid as a whole. pdl: may start while the previous kernel on the stream runs.
 nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16_t* q, const int32_t* sel,
@@ -391,6 +422,21 @@ nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16
   a.total_pages = (long long)n_groups(c) * c.slots;
   a.scale_log2 = c.scale * 1.4426950408889634f;
   a.sel_flag = ready;
+  if (c.stop_tau > 0.f) {
+    // early stop: one CTA per group, after the whole previous grid (no per-group flags)
+    StopArgs x;
+    x.scores = ws_at<float>(ws, w.scores);
+    x.tau = c.stop_tau;
+    x.used = ws_at<int32_t>(ws, w.used);
+    if (c.d == 128) {
+      if (c.block_size == 32) return launch_attn_stop_t<128, 32>(c, a, x, tk, tv, s, pdl);
+      if (c.block_size == 64) return launch_attn_stop_t<128, 64>(c, a, x, tk, tv, s, pdl);
+      return launch_attn_stop_t<128, 128>(c, a, x, tk, tv, s, pdl);
+    }
+    if (c.block_size == 32) return launch_attn_stop_t<64, 32>(c, a, x, tk, tv, s, pdl);
+    if (c.block_size == 64) return launch_attn_stop_t<64, 64>(c, a, x, tk, tv, s, pdl);
+    return launch_attn_stop_t<64, 128>(c, a, x, tk, tv, s, pdl);
+  }
   const bool finest = ready != nullptr && has_host(st);
   if (c.d == 128) {
     if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s, finest, pdl);
@@ -577,6 +623,7 @@ nosa_status nosa_decode_attn(const nosa_config* cfg, const nosa_state* st, const
   if ((r = check_state(c, st)) != NOSA_OK) return r;
   if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
   NOSA_CHECK(q && sel && out && aligned16(q) && aligned16(sel) && aligned16(out), "q/sel/out NULL or misaligned");
+  NOSA_CHECK(!(c.stop_tau > 0.f), "early stop visits blocks by the step's scores: use nosa_step");
   return launch_attn(c, st, q, sel, out, ws, as_stream(stream));
 }
 
@@ -616,7 +663,8 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   // (which themselves start on the group's published plan) have landed. With events each
   // kernel waits for the previous one as a whole, so that the events time kernels alone.
   const WsLayout w = ws_layout(c);
-  const bool flags = !events;
+  // early stop waits for the previous grid as a whole: no per-group flags then
+  const bool flags = !events && !(c.stop_tau > 0.f);
   a.sel_flag = flags ? ws_at<uint32_t>(ws, w.sel_flag) : nullptr;
   uint32_t* ready = !flags ? nullptr
                            : ws_at<uint32_t>(ws, has_host(st) ? w.copy_flag : w.sel_flag);
@@ -637,6 +685,7 @@ nosa_status nosa_plan_ahead(const nosa_config* cfg, const nosa_state* st, const 
   if ((r = check_state(c, st)) != NOSA_OK) return r;
   if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
   NOSA_CHECK(score_rows && evict && sel && miss_count, "plan_ahead buffer is NULL");
+  NOSA_CHECK(!(c.stop_tau > 0.f), "early stop is defined on the standard step order (nosa_step)");
   const void* ptrs[] = {score_rows, evict, sel, miss_count};
   for (const void* p : ptrs) NOSA_CHECK(aligned16(p), "plan_ahead buffer %p not 16-byte aligned", p);
   cudaStream_t s = as_stream(stream);
@@ -674,6 +723,7 @@ nosa_status nosa_attend(const nosa_config* cfg, const nosa_state* st, const uint
   if ((r = check_state(c, st)) != NOSA_OK) return r;
   if ((r = check_ws(c, ws, ws_bytes)) != NOSA_OK) return r;
   NOSA_CHECK(q && k_new && v_new && sel && out, "attend buffer is NULL");
+  NOSA_CHECK(!(c.stop_tau > 0.f), "early stop is defined on the standard step order (nosa_step)");
   const void* ptrs[] = {q, k_new, v_new, sel, out};
   for (const void* p : ptrs) NOSA_CHECK(aligned16(p), "attend buffer %p not 16-byte aligned", p);
   cudaStream_t s = as_stream(stream);
@@ -688,6 +738,18 @@ nosa_status nosa_attend(const nosa_config* cfg, const nosa_state* st, const uint
   NOSA_CUDA(cudaGetLastError());
   // no programmatic early start: the attention reads the length the append just wrote
   return launch_attn(c, st, q, sel, out, ws, s, ready, false);
+}
+
+nosa_status nosa_stop_counts(const nosa_config* cfg, const void* ws, size_t ws_bytes, int32_t* used,
+                             void* stream) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_ws(c, const_cast<void*>(ws), ws_bytes)) != NOSA_OK) return r;
+  NOSA_CHECK(used && aligned16(used), "used NULL or misaligned");
+  NOSA_CUDA(cudaMemcpyAsync(used, static_cast<const uint8_t*>(ws) + ws_layout(c).used,
+                            (size_t)c.B * c.Hq * 4, cudaMemcpyDeviceToDevice, as_stream(stream)));
+  return NOSA_OK;
 }
 
 nosa_status nosa_check_device(const nosa_state* st, void* stream, uint32_t* err_out) {
@@ -750,6 +812,7 @@ extern "C" nosa_status nosa_decode_attn_noalloc(const nosa_config* cfg, const no
   if ((r = check_state(c, st)) != NOSA_OK) return r;
   NOSA_CHECK(q && sel && out && aligned16(q) && aligned16(sel) && aligned16(out),
              "q/sel/out NULL or misaligned");
+  NOSA_CHECK(!(c.stop_tau > 0.f), "early stop visits blocks by the step's scores: use nosa_step");
   const size_t NG = n_groups(c);
   const size_t part_bytes = up256(NG * kPartialSlots * (size_t)(c.Hq / c.Hkv) * (c.d + 2) * 4);
   const size_t need = part_bytes + up256(NG * 4);

@@ -128,6 +128,7 @@ class NosaConfig:
     n_planted: int = 8
     plant_shift: float = 1.5
     score_mode: int = 0        # scoring variant bits: 1 overlapping windows, 2 per-row softmax
+    stop_tau: float = 0.0      # S2O early stop threshold on gain / mass (0: attend every block)
 
     @property
     def G(self) -> int:
@@ -235,6 +236,12 @@ def configs() -> dict:
     c["llama_softmax"] = c["llama"].with_(name="llama_softmax", score_mode=2, cfg_id=82)
     c["forecast_softmax"] = c["tiny_forecast"].with_(name="forecast_softmax", score_mode=2,
                                                      cfg_id=83)
+    # S2O early stop over the selected blocks, visited in decreasing block score
+    c["tiny_stop"] = c["tiny"].with_(name="tiny_stop", stop_tau=0.1, cfg_id=85)
+    c["tiny_dense_stop"] = c["tiny_dense"].with_(name="tiny_dense_stop", stop_tau=0.03, cfg_id=86)
+    c["ragged_stop"] = c["ragged_offload"].with_(name="ragged_stop", stop_tau=0.1, cfg_id=87)
+    c["llama_small_stop"] = c["llama_small"].with_(name="llama_small_stop", stop_tau=0.02, cfg_id=88)
+    c["llama_stop"] = c["llama"].with_(name="llama_stop", stop_tau=0.02, cfg_id=89)
     return c
 
 

@@ -31,6 +31,8 @@ _SRC = os.path.join(_HERE, "nosa_oracle.c")
 _SO = os.path.join(_HERE, "libnosa_oracle.so")
 
 MARGIN = 1e-3  # score margin required at the query-aware cut
+STOP_MARGIN = 1e-3   # early stop: relative distance of every gain/mass ratio from tau
+ORDER_MARGIN = 2e-5  # early stop: score gap between blocks adjacent in the visiting order
 
 
 def compile_oracle(src: str, out: str) -> str:
@@ -79,6 +81,8 @@ def load(path: Optional[str] = None):
         L.orc_residency.restype = ctypes.c_int
         L.orc_attend.argtypes = [vp, vp, vp, vp, vp]
         L.orc_attend.restype = None
+        L.orc_attend_stop.argtypes = [vp, vp, vp, vp, vp, ctypes.c_double, vp, vp, vp, vp]
+        L.orc_attend_stop.restype = None
         _libs[path] = L
     return _libs[path]
 
@@ -174,6 +178,20 @@ class Oracle:
                           _p(out))
         return out
 
+    def attend_stop(self, q, sel, scores, tau):
+        """S2O early-stop attention: (out, blocks used per head, decision margin per group,
+        order gap per group); see orc_attend_stop."""
+        c = self.cfg
+        NG = c.B * c.Hkv
+        out = np.empty((c.B, c.Hq, c.d), np.float64)
+        used = np.empty((c.B, c.Hq), np.int32)
+        mg, og = np.empty(NG), np.empty(NG)
+        self.L.orc_attend_stop(ctypes.byref(self.c), ctypes.byref(self.st),
+                               _p(np.ascontiguousarray(q)), _p(np.ascontiguousarray(sel, np.int32)),
+                               _p(np.ascontiguousarray(scores, np.float64)), float(tau), _p(out),
+                               _p(used), _p(mg), _p(og))
+        return out, used, mg, og
+
     def snapshot(self) -> dict:
         return {k: getattr(self, k).copy() for k in
                 ("len", "prev_sel", "alive", "block_slot", "slot_owner", "last_used")}
@@ -192,6 +210,7 @@ class StepRecord:
     out: np.ndarray             # fp64 [B][Hq][d]
     retries: np.ndarray         # int [B][Hkv]
     state: dict = field(default_factory=dict)
+    used: Optional[np.ndarray] = None   # int32 [B][Hq] blocks visited (early stop)
 
 
 @dataclass
@@ -237,6 +256,8 @@ def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = M
         raise ValueError("lookahead selection scores with the forecast row (n_score_rows == 1)")
     if lookahead and min(cfg.T) < 1:
         raise ValueError("lookahead needs a non-empty prefill")
+    if lookahead and cfg.stop_tau > 0:
+        raise ValueError("early stop is defined on the standard step order")
     inp = syn.make_inputs(cfg)
     # the oracle appends in place: inp.pool_k / pool_v rows >= T then hold the decode tokens
     orc = Oracle(cfg, inp.pool_k, inp.pool_v, inp.resident, lib_path, copy=False)
@@ -266,6 +287,11 @@ def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = M
             if cfg.score_mode & 2:
                 gap = _log_gap(scores, sel_t, src_t, gap)
             bad = (gap < margin) & (todo != 0)
+            if cfg.stop_tau > 0:
+                # early stop: every stop decision must sit clearly on one side of tau, and
+                # the visiting order must not hinge on near-equal scores
+                _, _, dm, og = orc.attend_stop(q16, sel_t, scores, cfg.stop_tau)
+                bad |= ((dm < STOP_MARGIN) | (og < ORDER_MARGIN)) & (todo != 0)
             if not bad.any():
                 break
             bad2 = bad.reshape(cfg.B, cfg.Hkv)
@@ -278,9 +304,13 @@ def run_case(cfg: syn.NosaConfig, steps: Optional[int] = None, margin: float = M
         miss = orc.residency(sel)
         if lookahead:
             orc.append(inp.k_new[t], inp.v_new[t])
-        out = orc.attend(q16, sel)
+        used = None
+        if cfg.stop_tau > 0:
+            out, used, _, _ = orc.attend_stop(q16, sel, scores, cfg.stop_tau)
+        else:
+            out = orc.attend(q16, sel)
         recs.append(StepRecord(q16, np.ascontiguousarray(rows), fc, scores, sel, src, gap, miss, out,
-                               retry, orc.snapshot() if keep_state else {}))
+                               retry, orc.snapshot() if keep_state else {}, used))
     case = Case(cfg, inp, recs)
     case.oracle = orc
     return case

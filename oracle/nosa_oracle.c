@@ -433,3 +433,99 @@ void orc_attend(const orc_cfg* c, const orc_state* st, const uint16_t* q, const 
     }
   }
 }
+
+/* S2O's monotone-gain early stop (gist.science/it/paper/2602.22575, "Regola di Arresto
+ * Anticipato"), applied to the selected blocks of a step. The blocks of S(t) are visited in
+ * decreasing block score (ties: lower index), the estimated importance, and every query
+ * head of the group runs the online softmax over them block by block. After block b the
+ * head's gain on b,
+ *     dl = sum over the tokens tau < L of b of exp(z_tau - m)     (m: running max after b)
+ * is compared with the accumulated mass l, which includes b: once dl < tau_stop * l the
+ * head stops (b is kept). o_h = acc / l at that point; tau_stop <= 0 never stops.
+ * used[b][h]: blocks the head visited. margin[gi]: the smallest |dl / l - tau_stop| / tau_stop
+ * over every decision taken in the group (INFINITY if none). order_gap[gi]: the smallest
+ * difference between the scores (their logs when score_mode has the softmax bit: those are
+ * probabilities) of consecutive blocks of the order, over the pairs that decide which
+ * blocks the heads visit (INFINITY if none). */
+void orc_attend_stop(const orc_cfg* c, const orc_state* st, const uint16_t* q, const int32_t* sel,
+                     const double* scores, double tau_stop, double* out, int32_t* used,
+                     double* margin, double* order_gap) {
+  const int NG = n_groups(c), G = c->Hq / c->Hkv, k = c->k_q + c->k_e, d = c->d;
+  const int nb = c->max_blocks;
+#pragma omp parallel for schedule(dynamic)
+  for (int gi = 0; gi < NG; ++gi) {
+    const int b = gi / c->Hkv, g = gi % c->Hkv;
+    const int L = st->len[gi];
+    orc_item* it = (orc_item*)malloc(sizeof(orc_item) * (size_t)(k + 1));
+    int n = 0;
+    for (int w = 0; w < k; ++w) {
+      const int j = sel[(size_t)gi * k + w];
+      if (j < 0) continue;
+      it[n].key = scores[(size_t)gi * nb + j];
+      it[n].idx = j;
+      ++n;
+    }
+    qsort(it, n, sizeof(orc_item), item_cmp);
+    double* acc = (double*)malloc(sizeof(double) * d);
+    double* zb = (double*)malloc(sizeof(double) * c->bs);
+    double mg = INFINITY;
+    int maxu = 0;
+    for (int r = 0; r < G; ++r) {
+      const int h = g * G + r;
+      const uint16_t* qh = q + ((size_t)b * c->Hq + h) * d;
+      double m = -INFINITY, l = 0.0;
+      for (int x = 0; x < d; ++x) acc[x] = 0.0;
+      int u = 0;
+      for (int p = 0; p < n; ++p) {
+        const int j = it[p].idx;
+        const int t0 = j * c->bs, t1 = ((j + 1) * c->bs < L) ? (j + 1) * c->bs : L;
+        double bm = -INFINITY;
+        for (int tau = t0; tau < t1; ++tau) {
+          const uint16_t* kt = st->K + tok_off(c, gi, tau);
+          double dot = 0.0;
+          for (int x = 0; x < d; ++x) dot += bf(qh[x]) * bf(kt[x]);
+          zb[tau - t0] = c->scale * dot;
+          if (zb[tau - t0] > bm) bm = zb[tau - t0];
+        }
+        const double m2 = (bm > m) ? bm : m;
+        const double rescale = (m == -INFINITY) ? 0.0 : exp(m - m2);
+        for (int x = 0; x < d; ++x) acc[x] *= rescale;
+        l *= rescale;
+        double dl = 0.0;
+        for (int tau = t0; tau < t1; ++tau) {
+          const double e = exp(zb[tau - t0] - m2);
+          const uint16_t* vt = st->V + tok_off(c, gi, tau);
+          dl += e;
+          for (int x = 0; x < d; ++x) acc[x] += e * bf(vt[x]);
+        }
+        l += dl;
+        m = m2;
+        ++u;
+        if (tau_stop > 0.0) {
+          const double ratio = dl / l;
+          const double rel = fabs(ratio - tau_stop) / tau_stop;
+          if (rel < mg) mg = rel;
+          if (ratio < tau_stop) break;
+        }
+      }
+      if (u > maxu) maxu = u;
+      used[(size_t)b * c->Hq + h] = u;
+      double* o = out + ((size_t)b * c->Hq + h) * d;
+      for (int x = 0; x < d; ++x) o[x] = (l > 0.0) ? acc[x] / l : 0.0;
+    }
+    /* positions 0 .. maxu-1 are visited by some head: the pairs (p, p+1) with p < maxu
+       (and p + 1 < n) decide which blocks those are */
+    double og = INFINITY;
+    if (tau_stop > 0.0)
+      for (int p = 0; p < maxu && p + 1 < n; ++p) {
+        const double gp = (c->score_mode & 2) ? log(it[p].key) - log(it[p + 1].key)
+                                              : it[p].key - it[p + 1].key;
+        if (gp < og) og = gp;
+      }
+    margin[gi] = mg;
+    order_gap[gi] = og;
+    free(zb);
+    free(acc);
+    free(it);
+  }
+}

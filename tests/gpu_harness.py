@@ -18,7 +18,8 @@ RTOL_L2 = 1e-3   # relative L2 error of the attention output vs fp64
 def c_config(cfg: syn.NosaConfig, attn_split: int = 0) -> nosa.nosa_config:
     return nosa.make_config(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.block, cfg.sub_block, cfg.k_q, cfg.k_e,
                             cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows,
-                            attn_split=attn_split, scale=cfg.scale, score_mode=cfg.score_mode)
+                            attn_split=attn_split, scale=cfg.scale, score_mode=cfg.score_mode,
+                            stop_tau=cfg.stop_tau)
 
 
 def dev(a: np.ndarray) -> torch.Tensor:
@@ -105,6 +106,11 @@ def compare_step(cache, cfg, rec, io: StepIO, t: int, check_state: bool = True):
     assert mx <= ATOL and rl2 <= RTOL_L2, f"{cfg.name} step {t}: max-abs {mx:.3g}, rel-L2 {rl2:.3g}"
     miss = io.miss.cpu().numpy()
     assert np.array_equal(miss, rec.miss), f"{cfg.name} step {t}: miss {miss} vs {rec.miss}"
+    if rec.used is not None:
+        used = torch.empty(cfg.B * cfg.Hq, dtype=torch.int32, device="cuda")
+        cache.stop_counts(used)
+        used = used.cpu().numpy().reshape(cfg.B, cfg.Hq)
+        assert np.array_equal(used, rec.used), f"{cfg.name} step {t}: blocks visited\n{used}\n{rec.used}"
     rc, err = cache.check()
     assert rc == nosa.NOSA_OK and err == 0, (rc, err)
     if check_state and rec.state:

@@ -342,6 +342,41 @@ def check_score_variants(cfg, lib_path=None, steps=2):
     return case
 
 
+def check_early_stop(cfg, lib_path=None, steps=None):
+    """S2O early stop against torch. Each group visits its selected blocks in decreasing
+    score (ties: lower index). For each head, with u = blocks it visited: every visited
+    block but the last gained at least tau of the mass accumulated up to it, the last gained
+    less (unless every block was visited); the gains and masses are torch logsumexp /
+    logcumsumexp of the token logits. The output is torch softmax attention over exactly
+    the visited blocks' tokens."""
+    case = O.run_case(cfg, steps=steps, lib_path=lib_path)
+    orc, c = case.oracle, case.cfg
+    tau = c.stop_tau
+    for t, rec in enumerate(case.steps):
+        for gi in range(c.B * c.Hkv):
+            b, g = gi // c.Hkv, gi % c.Hkv
+            Lt = c.T[b] + t + 1
+            blocks = [int(j) for j in rec.sel[gi] if j >= 0]
+            order = sorted(blocks, key=lambda j: (-rec.scores[gi][j], j))
+            K, V = _tokens(orc, gi, Lt)
+            Kt, Vt = torch.from_numpy(K), torch.from_numpy(V)
+            toks = [torch.arange(j * c.block, min((j + 1) * c.block, Lt)) for j in order]
+            for r in range(c.G):
+                h = g * c.G + r
+                u = int(rec.used[b, h])
+                assert 1 <= u <= len(order)
+                qh = torch.from_numpy(syn.bf16_to_f64(rec.q[b, h]))
+                lse = torch.stack([torch.logsumexp(c.scale * Kt[ix] @ qh, 0) for ix in toks])
+                cum = torch.logcumsumexp(lse, 0)
+                ratio = torch.exp(lse - cum).numpy()
+                assert np.all(ratio[:u - 1] >= tau), (t, gi, h, ratio[:u], tau)
+                assert u == len(order) or ratio[u - 1] < tau, (t, gi, h, ratio[:u], tau)
+                ix = torch.cat(toks[:u])
+                ref = (torch.softmax(c.scale * Kt[ix] @ qh, 0) @ Vt[ix]).numpy()
+                np.testing.assert_allclose(rec.out[b, h], ref, rtol=1e-11, atol=1e-13)
+    return case
+
+
 def run_all(lib_path=None):
     cs = syn.configs()
     check_topm_bruteforce(lib_path, trials=120)
@@ -351,6 +386,8 @@ def run_all(lib_path=None):
     check_attention_dense_sdpa(lib_path)
     for name in ("tiny_window", "ragged_window_softmax", "forecast_softmax", "ragged_window"):
         check_score_variants(cs[name], lib_path)
+    for name in ("tiny_stop", "ragged_stop"):
+        check_early_stop(cs[name], lib_path)
     for name in ("ragged", "tiny_forecast", "bs128_d64"):
         check_pooling_library(cs[name], lib_path, steps=2)
     for name in ("ragged", "ragged_offload", "g8"):

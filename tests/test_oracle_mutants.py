@@ -41,6 +41,12 @@ MUTANTS = {
         ("if (win && i + 1 < M) n1 =", "if (0 && win && i + 1 < M) n1 ="),
     "window weights its sub-blocks equally":
         ("kb[x] = (n0 * k0[x] + n1 * k1[x]) / (double)(n0 + n1);", "kb[x] = 0.5 * (k0[x] + k1[x]);"),
+    "early stop compares the gain with the mass before the block":
+        ("const double ratio = dl / l;", "const double ratio = dl / (l - dl + 1e-300);"),
+    "early stop visits the blocks in index order":
+        ("qsort(it, n, sizeof(orc_item), item_cmp);\n    double* acc", "(void)item_cmp;\n    double* acc"),
+    "early stop keeps going past the threshold":
+        ("if (ratio < tau_stop) break;", "if (ratio < 0.5 * tau_stop) break;"),
     "softmax without its normalizer":
         ("u += exp(z[(size_t)r * M + i] - mx[r]) / den[r];", "u += exp(z[(size_t)r * M + i] - mx[r]);"),
 }

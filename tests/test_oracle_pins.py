@@ -68,6 +68,11 @@ def test_score_variants_equal_torch_pooling(name):
     P.check_score_variants(CS[name])
 
 
+@pytest.mark.parametrize("name", ["tiny_stop", "tiny_dense_stop", "ragged_stop", "llama_small_stop"])
+def test_early_stop_equals_torch_rule(name):
+    P.check_early_stop(CS[name])
+
+
 def test_lookahead_dense_equals_sdpa():
     P.check_lookahead_dense_sdpa()
 
