@@ -54,7 +54,8 @@ def describe(cfg: syn.NosaConfig) -> str:
             f"block={cfg.block} sub_block={cfg.sub_block} k={cfg.k} (k_q={cfg.k_q}, k_e={cfg.k_e})"
             + (f" slots={cfg.slots} offload" if cfg.offload else " all KV in HBM")
             + (f" score_mode={cfg.score_mode}" if cfg.score_mode else "")
-            + (f" stop_tau={cfg.stop_tau}" if cfg.stop_tau else ""))
+            + (f" stop_tau={cfg.stop_tau}" if cfg.stop_tau else "")
+            + (" kc=bf16" if cfg.kc_bf16 else ""))
 
 
 def step_bytes(cfg: syn.NosaConfig, L: int, misses: int = 0, visited: float = None):
@@ -74,7 +75,7 @@ def step_bytes(cfg: syn.NosaConfig, L: int, misses: int = 0, visited: float = No
     # present tokens only when it is selected -- counted as full pages otherwise
     kv = nsel * bs * d * 2 * 2
     attn = NG * (kv + G * d * 2 + G * d * 4 + cfg.k * 4 + cfg.k * 4)
-    score = NG * (M * d * 4 + N * 4 + 2 * 2 * 4 * (-(-N // 32)) + cfg.rows * d * 2
+    score = NG * (M * d * (2 if cfg.kc_bf16 else 4) + N * 4 + 2 * 2 * 4 * (-(-N // 32)) + cfg.rows * d * 2
                   + 2 * d * 2 + N * 4 * 2 + cfg.k * 4)
     page = bs * d * 2
     return attn + score + misses * 2 * page, attn, score, misses * 2 * page
@@ -260,7 +261,7 @@ def run_gpu(args, cfg):
     NG = cfg.B * cfg.Hkv
     cc = nosa.make_config(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.block, cfg.sub_block, cfg.k_q, cfg.k_e,
                           cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows, scale=cfg.scale, score_mode=cfg.score_mode,
-                          stop_tau=cfg.stop_tau)
+                          stop_tau=cfg.stop_tau, kc_bf16=cfg.kc_bf16)
     cache = nosa.NosaCache(cc, offload=cfg.offload)
     pk = torch.from_numpy(inp.pool_k.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)
     pv = torch.from_numpy(inp.pool_v.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)

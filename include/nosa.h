@@ -86,6 +86,9 @@ typedef struct nosa_config {
                              stops after the first block whose gain in softmax mass is below
                              stop_tau times the mass accumulated so far, that block included.
                              0: attend every selected block. Needs k <= 1024. */
+  int32_t kc_bf16;        /* 1: state->kc holds bf16 sub-block means (each mean is summed in fp32 in
+                             token order, divided in fp32 and rounded to nearest even), half the
+                             score kernel's bytes; 0: fp32 means. */
 } nosa_config;
 
 #define NOSA_SCORE_WINDOW 1
@@ -101,7 +104,7 @@ typedef struct nosa_config {
  */
 typedef struct nosa_state {
   int32_t* seq_len;       /* [B*Hkv] tokens in the cache */
-  float* kc;              /* [B*Hkv][max_sub][d] fp32 sub-block mean keys */
+  float* kc;              /* [B*Hkv][max_sub][d] sub-block mean keys: fp32, or bf16 with kc_bf16 */
   uint32_t* prev_sel;     /* [B*Hkv][W] bitmask of S(t-1) */
   uint32_t* alive;        /* [B*Hkv][W] bitmask of A(t-1), blocks still eligible for Gamma_e */
   int32_t* last_used;     /* [B*Hkv][max_blocks] context length when last needed (LRU stamp) */

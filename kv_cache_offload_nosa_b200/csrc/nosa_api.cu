@@ -70,6 +70,7 @@ nosa_status check_cfg(const nosa_config* cp) {
   NOSA_CHECK(!(c.score_mode & NOSA_SCORE_SOFTMAX) || c.n_score_rows <= kMaxSoftRows,
              "softmax scoring supports at most %d scoring rows", kMaxSoftRows);
   NOSA_CHECK(c.stop_tau >= 0.f && c.stop_tau < 1e30f, "stop_tau must be >= 0 and finite");
+  NOSA_CHECK(c.kc_bf16 == 0 || c.kc_bf16 == 1, "kc_bf16 must be 0 or 1");
   NOSA_CHECK(!(c.stop_tau > 0.f) || kk(c) <= kStopMaxK, "early stop supports k <= %d", kStopMaxK);
   NOSA_CHECK(c.scale > 0.f, "scale must be > 0");
   const long long groups = (long long)c.B * c.Hkv;
@@ -158,6 +159,7 @@ StepArgs step_args(const nosa_config& c, const nosa_state* st) {
   StepArgs a;
   memset(&a, 0, sizeof(a));
   a.kc = st->kc;
+  a.kc16 = c.kc_bf16;
   a.seq_len = st->seq_len;
   a.max_blocks = c.max_blocks;
   a.max_sub = max_sub(c);
@@ -193,36 +195,30 @@ void set_ws(StepArgs& a, const nosa_config& c, void* ws) {
 }
 
 // ------------------------------------------------------------------ launches
-template <int D, bool FUSED, int VARIANT>
+template <int D, bool FUSED, int VARIANT, bool KC16>
 nosa_status launch_score_t(const nosa_config& c, const StepArgs& a, cudaStream_t s) {
   dim3 grid((max_sub(c) + kChunkSub - 1) / kChunkSub, n_groups(c));
   const size_t dsm = FUSED ? sel_smem_bytes(c.max_blocks) : 0;
-  auto k = score_kernel<D, FUSED, VARIANT>;
+  auto k = score_kernel<D, FUSED, VARIANT, KC16>;
   if (dsm > 48 * 1024) NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm));
   k<<<grid, kScoreThreads, dsm, s>>>(a);
   NOSA_CUDA(cudaGetLastError());
   return NOSA_OK;
 }
 
+template <int D, bool FUSED, int VARIANT>
+nosa_status launch_score_kc(const nosa_config& c, const StepArgs& a, cudaStream_t s) {
+  return c.kc_bf16 ? launch_score_t<D, FUSED, VARIANT, true>(c, a, s)
+                   : launch_score_t<D, FUSED, VARIANT, false>(c, a, s);
+}
+
 template <bool FUSED>
 nosa_status launch_score(const nosa_config& c, const StepArgs& a, cudaStream_t s) {
   if (FUSED && (c.score_mode & NOSA_SCORE_SOFTMAX))
-    return c.d == 128 ? launch_score_t<128, true, 2>(c, a, s) : launch_score_t<64, true, 2>(c, a, s);
+    return c.d == 128 ? launch_score_kc<128, true, 2>(c, a, s) : launch_score_kc<64, true, 2>(c, a, s);
   if (FUSED && c.score_mode)
-    return c.d == 128 ? launch_score_t<128, true, 1>(c, a, s) : launch_score_t<64, true, 1>(c, a, s);
-  dim3 grid((max_sub(c) + kChunkSub - 1) / kChunkSub, n_groups(c));
-  const size_t dsm = FUSED ? sel_smem_bytes(c.max_blocks) : 0;
-  if (c.d == 128) {
-    auto k = score_kernel<128, FUSED>;
-    if (dsm > 48 * 1024) NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm));
-    k<<<grid, kScoreThreads, dsm, s>>>(a);
-  } else {
-    auto k = score_kernel<64, FUSED>;
-    if (dsm > 48 * 1024) NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm));
-    k<<<grid, kScoreThreads, dsm, s>>>(a);
-  }
-  NOSA_CUDA(cudaGetLastError());
-  return NOSA_OK;
+    return c.d == 128 ? launch_score_kc<128, true, 1>(c, a, s) : launch_score_kc<64, true, 1>(c, a, s);
+  return c.d == 128 ? launch_score_kc<128, FUSED, 0>(c, a, s) : launch_score_kc<64, FUSED, 0>(c, a, s);
 }
 
 nosa_status launch_sel_kernel(void (*k)(StepArgs), const nosa_config& c, const StepArgs& a,
@@ -474,7 +470,7 @@ nosa_status nosa_state_sizes(const nosa_config* cfg, nosa_sizes* out) {
   const nosa_config& c = *cfg;
   const size_t NG = n_groups(c);
   out->seq_len = NG * 4;
-  out->kc = NG * max_sub(c) * (size_t)c.d * 4;
+  out->kc = NG * max_sub(c) * (size_t)c.d * (c.kc_bf16 ? 2 : 4);
   out->prev_sel = NG * words(c) * 4;
   out->alive = NG * words(c) * 4;
   out->last_used = NG * c.max_blocks * 4;
@@ -538,9 +534,11 @@ nosa_status nosa_state_init(const nosa_config* cfg, const nosa_state* st, const 
   const int subs = 256 / c.d * 4;
   dim3 g((max_sub(c) + subs - 1) / subs, n_groups(c));
   if (c.d == 128)
-    init_kc_kernel<128><<<g, 256, 0, s>>>(prefill_len, c.Hkv, src, ppg, st->kc, max_sub(c), c.block_size, c.sub_block);
+    if (c.kc_bf16) init_kc_kernel<128, true><<<g, 256, 0, s>>>(prefill_len, c.Hkv, src, ppg, st->kc, max_sub(c), c.block_size, c.sub_block);
+    else init_kc_kernel<128, false><<<g, 256, 0, s>>>(prefill_len, c.Hkv, src, ppg, st->kc, max_sub(c), c.block_size, c.sub_block);
   else
-    init_kc_kernel<64><<<g, 256, 0, s>>>(prefill_len, c.Hkv, src, ppg, st->kc, max_sub(c), c.block_size, c.sub_block);
+    if (c.kc_bf16) init_kc_kernel<64, true><<<g, 256, 0, s>>>(prefill_len, c.Hkv, src, ppg, st->kc, max_sub(c), c.block_size, c.sub_block);
+    else init_kc_kernel<64, false><<<g, 256, 0, s>>>(prefill_len, c.Hkv, src, ppg, st->kc, max_sub(c), c.block_size, c.sub_block);
   NOSA_CUDA(cudaGetLastError());
   if (has_host(st)) return launch_copy(c, st, ws, s);
   return NOSA_OK;

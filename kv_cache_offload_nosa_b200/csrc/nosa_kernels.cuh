@@ -9,6 +9,8 @@
 // the dual selection and, with host pools, the residency plan.
 #pragma once
 
+#include <type_traits>
+
 #include "nosa_select.cuh"
 
 namespace nosa {
@@ -54,6 +56,7 @@ struct StepArgs {
   int append;             // fused score kernel: 1 appends the step's token first, 0 scores the
                           // cache as it stands (lookahead planning)
   const uint32_t* ready;  // append_kernel: per-group flags to acquire before writing, or NULL
+  int kc16;               // kc holds bf16 means (else fp32)
   int mode;               // scoring variant bits (1 windows, 2 per-row softmax); 0 = NOSA pool
   float* units;           // variants: per-sub-block values [B*Hkv][rows][max_sub] (workspace)
 };
@@ -176,16 +179,21 @@ __device__ void append_token(const StepArgs& a, int gi, int len0) {
       a.host_k[(hbase + r) * D + x] = kx;
       a.host_v[(hbase + r) * D + x] = vx;
     }
-    a.kc[((size_t)gi * a.max_sub + sb) * D + x] = __fdiv_rn(sum, (float)(pos - t0 + 1));
+    const float mean = __fdiv_rn(sum, (float)(pos - t0 + 1));
+    const size_t ki = ((size_t)gi * a.max_sub + sb) * D + x;
+    if (a.kc16) reinterpret_cast<__nv_bfloat16*>(a.kc)[ki] = __float2bfloat16_rn(mean);
+    else a.kc[ki] = mean;
   }
 }
 
 // VARIANT: the scoring variants (a.mode != 0; 1: mean of the rows, windows; 2: per-row
 // softmax); the chunks leave per-sub-block values in a.units and the group's last CTA turns
 // them into block scores (fused launches only).
-template <int D, bool FUSED, int VARIANT = 0>
+// KC16: kc holds bf16 means (one 16-byte load carries 8 of them; the lanes of a sub-block row
+// still read it in contiguous 128-byte pieces).
+template <int D, bool FUSED, int VARIANT = 0, bool KC16 = false>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
-  constexpr int LPS = D / 16;        // lanes per sub-block (16 floats each)
+  constexpr int LPS = D / 16;        // lanes per sub-block (16 values each)
   constexpr int SPW = 32 / LPS;      // sub-blocks per warp pass
   constexpr int PASS = SPW * (kScoreThreads / 32);
   __shared__ float qbar[D];
@@ -198,20 +206,27 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   const int gi = blockIdx.y, c = blockIdx.x;
   const int i0 = c * kChunkSub;
   const int sub = lane / LPS, part = lane % LPS;
-  const float4* kcg = reinterpret_cast<const float4*>(a.kc + (size_t)gi * a.max_sub * D);
+  using Vec = typename std::conditional<KC16, uint4, float4>::type;
+  constexpr int NV = KC16 ? 2 : 4;          // 16-byte loads per lane and sub-block row
+  constexpr int EV = KC16 ? 8 : 4;          // values per 16-byte load
+  constexpr int VPR = D / EV;               // 16-byte vectors per row
+  const Vec* kcg = reinterpret_cast<const Vec*>(
+      reinterpret_cast<const uint8_t*>(a.kc) + (size_t)gi * a.max_sub * D * (KC16 ? 2 : 4));
 
   if (FUSED) griddep_launch_dependents();  // the next kernel may start its prologue
   // first batch of kc loads goes out before anything that depends on seq_len
   const int icap = min(i0 + kChunkSub, a.max_sub);
   int base = i0 + warp * SPW;
-  float4 va[4], vb[4];
-  auto load_batch = [&](int bse, int lim, float4* xa, float4* xb) {
+  Vec va[NV], vb[NV];
+  auto load_batch = [&](int bse, int lim, Vec* xa, Vec* xb) {
     const int ia = bse + sub, ib = bse + PASS + sub;
+    Vec z;
+    memset(&z, 0, sizeof(z));
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
+    for (int jj = 0; jj < NV; ++jj) {
       const int p4 = part + LPS * jj;
-      xa[jj] = (ia < lim) ? __ldcs(kcg + (size_t)ia * (D / 4) + p4) : make_float4(0, 0, 0, 0);
-      xb[jj] = (ib < lim) ? __ldcs(kcg + (size_t)ib * (D / 4) + p4) : make_float4(0, 0, 0, 0);
+      xa[jj] = (ia < lim) ? __ldcs(kcg + (size_t)ia * VPR + p4) : z;
+      xb[jj] = (ib < lim) ? __ldcs(kcg + (size_t)ib * VPR + p4) : z;
     }
   };
   load_batch(base, icap, va, vb);
@@ -269,7 +284,16 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
 #pragma unroll
       for (int f = 0; f < RF; ++f) {
         const int i = b0 + f * WROWS + sub2;
-        x[f] = (i < i1) ? __ldcs(kcg + (size_t)i * (D / 4) + p2) : make_float4(0, 0, 0, 0);
+        x[f] = make_float4(0, 0, 0, 0);
+        if (i < i1) {
+          if constexpr (KC16) {
+            const uint2 w = __ldcs(reinterpret_cast<const uint2*>(kcg) + (size_t)i * (D / 4) + p2);
+            x[f] = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                               __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+          } else {
+            x[f] = __ldcs(reinterpret_cast<const float4*>(kcg) + (size_t)i * (D / 4) + p2);
+          }
+        }
       }
 #pragma unroll
       for (int r = 0; r < kMaxSoftRows; ++r) {
@@ -292,28 +316,40 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
     }
   }
   if (!soft && i0 < i1) {
-    float qr[16];
+    float qr[16];  // this lane's 16 values of qbar, in the order of its loads
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
+    for (int jj = 0; jj < NV; ++jj) {
       const int p4 = part + LPS * jj;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) qr[4 * jj + e] = qbar[4 * p4 + e];
+      for (int e = 0; e < EV; ++e) qr[EV * jj + e] = qbar[EV * p4 + e];
     }
     for (; base < i1; base += 2 * PASS) {
-      float4 na[4], nb[4];
+      Vec na[NV], nb[NV];
       load_batch(base + 2 * PASS, i1, na, nb);  // next batch in flight during this one
       const int ia = base + sub, ib = base + PASS + sub;
       float da = 0.f, db = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        da = fmaf(qr[4 * jj + 0], va[jj].x, da);
-        da = fmaf(qr[4 * jj + 1], va[jj].y, da);
-        da = fmaf(qr[4 * jj + 2], va[jj].z, da);
-        da = fmaf(qr[4 * jj + 3], va[jj].w, da);
-        db = fmaf(qr[4 * jj + 0], vb[jj].x, db);
-        db = fmaf(qr[4 * jj + 1], vb[jj].y, db);
-        db = fmaf(qr[4 * jj + 2], vb[jj].z, db);
-        db = fmaf(qr[4 * jj + 3], vb[jj].w, db);
+      for (int jj = 0; jj < NV; ++jj) {
+        if constexpr (KC16) {
+          const uint32_t wa[4] = {va[jj].x, va[jj].y, va[jj].z, va[jj].w};
+          const uint32_t wb[4] = {vb[jj].x, vb[jj].y, vb[jj].z, vb[jj].w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            da = fmaf(qr[8 * jj + 2 * h], __uint_as_float(wa[h] << 16), da);
+            da = fmaf(qr[8 * jj + 2 * h + 1], __uint_as_float(wa[h] & 0xffff0000u), da);
+            db = fmaf(qr[8 * jj + 2 * h], __uint_as_float(wb[h] << 16), db);
+            db = fmaf(qr[8 * jj + 2 * h + 1], __uint_as_float(wb[h] & 0xffff0000u), db);
+          }
+        } else {
+          da = fmaf(qr[4 * jj + 0], va[jj].x, da);
+          da = fmaf(qr[4 * jj + 1], va[jj].y, da);
+          da = fmaf(qr[4 * jj + 2], va[jj].z, da);
+          da = fmaf(qr[4 * jj + 3], va[jj].w, da);
+          db = fmaf(qr[4 * jj + 0], vb[jj].x, db);
+          db = fmaf(qr[4 * jj + 1], vb[jj].y, db);
+          db = fmaf(qr[4 * jj + 2], vb[jj].z, db);
+          db = fmaf(qr[4 * jj + 3], vb[jj].w, db);
+        }
       }
 #pragma unroll
       for (int o = LPS / 2; o >= 1; o >>= 1) {
@@ -325,7 +361,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
         if (ib < i1) su[ib - i0] = db;
       }
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
+      for (int jj = 0; jj < NV; ++jj) {
         va[jj] = na[jj];
         vb[jj] = nb[jj];
       }
@@ -626,8 +662,9 @@ __global__ void __launch_bounds__(256) init_tables_kernel(InitArgs a) {
   if (tid == 0) a.copy_count[gi] = total < a.slots ? total : a.slots;
 }
 
-// kc[i] = fp32 mean of the present tokens of sub-block i (prefill), zero past the prefill.
-template <int D>
+// kc[i] = mean of the present tokens of sub-block i (prefill; fp32, or rounded to bf16 with
+// KC16), zero past the prefill.
+template <int D, bool KC16>
 __global__ void __launch_bounds__(256) init_kc_kernel(const int32_t* prefill_len, int Hkv,
                                                       const uint16_t* src, int src_pages_per_group,
                                                       float* kc, int max_sub, int bs, int s) {
@@ -643,7 +680,10 @@ __global__ void __launch_bounds__(256) init_kc_kernel(const int32_t* prefill_len
       const int j = tau / bs, r = tau % bs;
       sum += bf16_bits_to_f32(src[(((size_t)gi * src_pages_per_group + j) * bs + r) * D + x]);
     }
-    kc[((size_t)gi * max_sub + i) * D + x] = (t1 > t0) ? __fdiv_rn(sum, (float)(t1 - t0)) : 0.f;
+    const float mean = (t1 > t0) ? __fdiv_rn(sum, (float)(t1 - t0)) : 0.f;
+    const size_t ki = ((size_t)gi * max_sub + i) * D + x;
+    if (KC16) reinterpret_cast<__nv_bfloat16*>(kc)[ki] = __float2bfloat16_rn(mean);
+    else kc[ki] = mean;
   }
 }
 

@@ -129,6 +129,7 @@ class NosaConfig:
     plant_shift: float = 1.5
     score_mode: int = 0        # scoring variant bits: 1 overlapping windows, 2 per-row softmax
     stop_tau: float = 0.0      # S2O early stop threshold on gain / mass (0: attend every block)
+    kc_bf16: int = 0           # 1: sub-block mean keys stored as bf16
 
     @property
     def G(self) -> int:
@@ -242,6 +243,13 @@ def configs() -> dict:
     c["ragged_stop"] = c["ragged_offload"].with_(name="ragged_stop", stop_tau=0.1, cfg_id=87)
     c["llama_small_stop"] = c["llama_small"].with_(name="llama_small_stop", stop_tau=0.02, cfg_id=88)
     c["llama_stop"] = c["llama"].with_(name="llama_stop", stop_tau=0.02, cfg_id=89)
+    # bf16 sub-block mean keys (half the score kernel's bytes)
+    c["tiny_kc16"] = c["tiny"].with_(name="tiny_kc16", kc_bf16=1, cfg_id=93)
+    c["ragged_kc16"] = c["ragged_offload"].with_(name="ragged_kc16", kc_bf16=1, cfg_id=94)
+    c["llama_small_kc16"] = c["llama_small"].with_(name="llama_small_kc16", kc_bf16=1, cfg_id=95)
+    c["g8_kc16"] = c["g8"].with_(name="g8_kc16", kc_bf16=1, score_mode=3, cfg_id=96)
+    c["bs128_d64_kc16"] = c["bs128_d64"].with_(name="bs128_d64_kc16", kc_bf16=1, cfg_id=97)
+    c["llama_kc16"] = c["llama"].with_(name="llama_kc16", kc_bf16=1, cfg_id=98)
     return c
 
 

@@ -50,7 +50,7 @@ def build(force: bool = False) -> str:
 class OrcCfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "Hq", "Hkv", "d", "bs", "s", "k_q", "k_e", "n_rows", "max_blocks", "slots",
-                 "offload", "score_mode")] + [("scale", ctypes.c_double)]
+                 "offload", "score_mode", "kc_bf16")] + [("scale", ctypes.c_double)]
 
 
 class OrcState(ctypes.Structure):
@@ -113,7 +113,7 @@ class Oracle:
         c = cfg
         NG, nb = c.B * c.Hkv, c.max_blocks
         self.c = OrcCfg(c.B, c.Hq, c.Hkv, c.d, c.block, c.sub_block, c.k_q, c.k_e, c.rows, nb,
-                        c.n_slots, int(c.offload), int(c.score_mode), c.scale)
+                        c.n_slots, int(c.offload), int(c.score_mode), int(c.kc_bf16), c.scale)
         # copy=False: the oracle appends into the caller's arrays (rows >= T change)
         self.K = np.ascontiguousarray(pool_k)
         self.V = np.ascontiguousarray(pool_v)

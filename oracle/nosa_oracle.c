@@ -60,6 +60,7 @@ typedef struct {
   int32_t slots;          /* HBM slots per group (offload model) */
   int32_t offload;        /* 1: model HBM residency */
   int32_t score_mode;     /* scoring variant bits, see orc_block_scores (0: the NOSA pool) */
+  int32_t kc_bf16;        /* 1: sub-block means stored as bf16 (see sub_mean) */
   double scale;           /* sigma = 1/sqrt(d) */
 } orc_cfg;
 
@@ -91,12 +92,33 @@ static size_t tok_off(const orc_cfg* c, int gi, int tau) {
 }
 
 /* Mean key of sub-block i over its present tokens (fp64). */
+/* bf16 bit pattern of a finite float, rounded to nearest, ties to even (the definition:
+ * add half of the dropped part's unit, plus one when the kept part is odd, then truncate). */
+static uint16_t bf16_rne(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+/* Mean key of sub-block i over its present tokens. fp64, or with kc_bf16 the value a bf16
+ * store of the mean holds: the kernels sum the bf16 tokens in fp32 in token order, divide in
+ * fp32 (correctly rounded) and round to bf16 (nearest, ties to even); the oracle takes that
+ * quantisation the same way so that both sides hold the same codes. */
 static void sub_mean(const orc_cfg* c, const orc_state* st, int gi, int i, double* out) {
   const int L = st->len[gi];
   const int t0 = i * c->s;
   const int t1 = (t0 + c->s < L) ? t0 + c->s : L;
   for (int x = 0; x < c->d; ++x) out[x] = 0.0;
   if (t1 <= t0) return;
+  if (c->kc_bf16) {
+    for (int x = 0; x < c->d; ++x) {
+      float sum = 0.0f;
+      for (int tau = t0; tau < t1; ++tau) sum += (float)bf(st->K[tok_off(c, gi, tau) + x]);
+      out[x] = bf((uint16_t)bf16_rne(sum / (float)(t1 - t0)));
+    }
+    return;
+  }
   for (int tau = t0; tau < t1; ++tau) {
     const uint16_t* k = st->K + tok_off(c, gi, tau);
     for (int x = 0; x < c->d; ++x) out[x] += bf(k[x]);

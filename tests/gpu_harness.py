@@ -19,7 +19,7 @@ def c_config(cfg: syn.NosaConfig, attn_split: int = 0) -> nosa.nosa_config:
     return nosa.make_config(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.block, cfg.sub_block, cfg.k_q, cfg.k_e,
                             cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows,
                             attn_split=attn_split, scale=cfg.scale, score_mode=cfg.score_mode,
-                            stop_tau=cfg.stop_tau)
+                            stop_tau=cfg.stop_tau, kc_bf16=cfg.kc_bf16)
 
 
 def dev(a: np.ndarray) -> torch.Tensor:

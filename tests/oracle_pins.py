@@ -377,6 +377,34 @@ def check_early_stop(cfg, lib_path=None, steps=None):
     return case
 
 
+def check_kc_bf16(cfg, lib_path=None, steps=2):
+    """bf16 sub-block means: every stored code equals numpy's -- the sequential fp32 sum of the
+    sub-block's bf16 tokens (cumsum), divided in fp32, rounded to nearest even bf16 -- bit
+    for bit, and the block scores are the two-stage pool of those codes."""
+    case = O.run_case(cfg, steps=steps, lib_path=lib_path)
+    orc, c = case.oracle, case.cfg
+    s, spb = c.sub_block, c.block // c.sub_block
+    t = len(case.steps) - 1
+    rec = case.steps[t]
+    for gi in range(c.B * c.Hkv):
+        b, g = gi // c.Hkv, gi % c.Hkv
+        Lt = c.T[b] + t + 1
+        M, N = -(-Lt // s), -(-Lt // c.block)
+        Kb = orc.K[b, g, :Lt].view(np.uint16)
+        K32 = syn.bf16_to_f64(Kb).astype(np.float32)
+        want = np.empty((M, c.d), np.float64)
+        for i in range(M):
+            t0, t1 = i * s, min((i + 1) * s, Lt)
+            tot = np.cumsum(K32[t0:t1], axis=0, dtype=np.float32)[-1]
+            want[i] = syn.bf16_to_f64(syn.round_bf16((tot / np.float32(t1 - t0)).astype(np.float64)))
+        np.testing.assert_array_equal(orc.kbar[gi, :M], want)
+        rows = syn.bf16_to_f64(rec.rows[b, g] if c.n_score_rows == 1 else rec.q[b, g * c.G:(g + 1) * c.G])
+        u = (c.scale * rows.reshape(-1, c.d) @ want.T).mean(0)
+        blk = np.array([u[j * spb:min((j + 1) * spb, M)].max() for j in range(N)])
+        np.testing.assert_allclose(rec.scores[gi][:N], blk, rtol=1e-12, atol=1e-14)
+    return case
+
+
 def run_all(lib_path=None):
     cs = syn.configs()
     check_topm_bruteforce(lib_path, trials=120)
@@ -388,6 +416,8 @@ def run_all(lib_path=None):
         check_score_variants(cs[name], lib_path)
     for name in ("tiny_stop", "ragged_stop"):
         check_early_stop(cs[name], lib_path)
+    for name in ("tiny_kc16", "ragged_kc16"):
+        check_kc_bf16(cs[name], lib_path)
     for name in ("ragged", "tiny_forecast", "bs128_d64"):
         check_pooling_library(cs[name], lib_path, steps=2)
     for name in ("ragged", "ragged_offload", "g8"):

@@ -45,7 +45,8 @@ def cfg(**kw):
                                  dict(Hq=12, Hkv=4, ), dict(Hq=7), dict(k_q=0, k_e=0),
                                  dict(k_q=30, k_e=20), dict(max_blocks=9000), dict(slots=0),
                                  dict(n_score_rows=2), dict(scale=0.0), dict(sub_block=128),
-                                 dict(score_mode=4), dict(score_mode=-1)])
+                                 dict(score_mode=4), dict(score_mode=-1), dict(kc_bf16=2),
+                                 dict(stop_tau=-1.0)])
 def test_bad_config_is_rejected_on_host(lib, bad):
     c = cfg(**bad)
     n = ctypes.c_size_t()
@@ -75,6 +76,10 @@ def test_score_variants_reserve_their_values(lib):
     assert win - base >= NG * max_sub * 4
     assert soft - base >= NG * 4 * max_sub * 4      # G = 4 rows
     assert nosa.workspace_size(cfg(score_mode=3, n_score_rows=1)) - base >= NG * max_sub * 4
+
+
+def test_bf16_kc_halves_its_buffer(lib):
+    assert nosa.state_sizes(cfg(kc_bf16=1)).kc * 2 == nosa.state_sizes(cfg()).kc
 
 
 def test_status_strings(lib):

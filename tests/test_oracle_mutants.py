@@ -47,6 +47,8 @@ MUTANTS = {
         ("qsort(it, n, sizeof(orc_item), item_cmp);\n    double* acc", "(void)item_cmp;\n    double* acc"),
     "early stop keeps going past the threshold":
         ("if (ratio < tau_stop) break;", "if (ratio < 0.5 * tau_stop) break;"),
+    "bf16 means truncated instead of rounded":
+        ("u += 0x7FFFu + ((u >> 16) & 1u);", "u += 0u;"),
     "softmax without its normalizer":
         ("u += exp(z[(size_t)r * M + i] - mx[r]) / den[r];", "u += exp(z[(size_t)r * M + i] - mx[r]);"),
 }

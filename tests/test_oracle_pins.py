@@ -73,6 +73,11 @@ def test_early_stop_equals_torch_rule(name):
     P.check_early_stop(CS[name])
 
 
+@pytest.mark.parametrize("name", ["tiny_kc16", "ragged_kc16", "llama_small_kc16", "bs128_d64_kc16"])
+def test_kc_bf16_codes_equal_numpy(name):
+    P.check_kc_bf16(CS[name])
+
+
 def test_lookahead_dense_equals_sdpa():
     P.check_lookahead_dense_sdpa()
 
