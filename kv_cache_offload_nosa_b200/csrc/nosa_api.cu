@@ -418,6 +418,7 @@ nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16
   a.total_pages = (long long)n_groups(c) * c.slots;
   a.scale_log2 = c.scale * 1.4426950408889634f;
   a.sel_flag = ready;
+  a.identity = !has_host(st);
   if (c.stop_tau > 0.f) {
     // early stop: one CTA per group, after the whole previous grid (no per-group flags)
     StopArgs x;

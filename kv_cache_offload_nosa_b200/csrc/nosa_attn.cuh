@@ -43,6 +43,8 @@ struct AttnArgs {
   long long total_pages;
   float scale_log2;           // sigma * log2(e)
   uint32_t* sel_flag;         // [B*Hkv * kFlagStride] per-group "ready" flags, or NULL
+  int identity;               // no host pools: block j of group g is page g * max_blocks + j
+                              // (the state's block table is that identity), so no lookup
 };
 
 struct TaskInfo {
@@ -140,7 +142,8 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
           j_l = -1;
         }
         if (j_l >= 0) {
-          page_l = __ldcg(a.block_table + (size_t)gi_l * a.max_blocks + j_l);
+          page_l = a.identity ? gi_l * a.max_blocks + j_l
+                              : __ldcg(a.block_table + (size_t)gi_l * a.max_blocks + j_l);
           if (page_l < 0 || page_l >= a.total_pages) {
             set_err(a.err, NOSA_ERR_BLOCK_TABLE);
             j_l = -1;
