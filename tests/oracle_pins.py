@@ -190,8 +190,8 @@ def check_hand_dual_selection(lib_path=None):
         assert [j for j in range(N) if orc.alive[0, j]] == h["expect_alive_below_N"][t]
 
 
-def check_hand_residency(lib_path=None):
-    h = json.load(open(os.path.join(GOLDEN, "hand_residency.json")))
+def check_hand_residency(lib_path=None, name="hand_residency.json"):
+    h = json.load(open(os.path.join(GOLDEN, name)))
     cfg = _hand_cfg(h)
     nb = cfg.max_blocks
     z = np.zeros((1, 1, nb * cfg.block, cfg.d), np.uint16)
@@ -410,6 +410,7 @@ def run_all(lib_path=None):
     check_topm_bruteforce(lib_path, trials=120)
     check_hand_dual_selection(lib_path)
     check_hand_residency(lib_path)
+    check_hand_residency(lib_path, "hand_residency_order.json")
     check_static_closed_form(lib_path)
     check_attention_dense_sdpa(lib_path)
     for name in ("tiny_window", "ragged_window_softmax", "forecast_softmax", "ragged_window"):
@@ -420,7 +421,7 @@ def run_all(lib_path=None):
         check_kc_bf16(cs[name], lib_path)
     for name in ("ragged", "tiny_forecast", "bs128_d64"):
         check_pooling_library(cs[name], lib_path, steps=2)
-    for name in ("ragged", "ragged_offload", "g8"):
+    for name in ("ragged", "ragged_offload", "g8", "short_kq0"):
         case = check_attention_subset(cs[name], lib_path)
         check_selection_trace(case)
         if case.cfg.offload:

@@ -14,7 +14,8 @@ pytestmark = pytest.mark.gpu
 
 CS = syn.configs()
 SMALL = ["tiny", "tiny_dense", "tiny_static", "tiny_forecast", "llama_small", "offload_small",
-         "sink_small", "ragged", "ragged_offload", "empty", "bs128_d64", "g8"]
+         "sink_small", "ragged", "ragged_offload", "empty", "bs128_d64", "g8", "short_kq0",
+         "short_kq0_offload"]
 
 _cases = {}
 

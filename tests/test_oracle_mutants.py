@@ -51,6 +51,48 @@ MUTANTS = {
         ("u += 0x7FFFu + ((u >> 16) & 1u);", "u += 0u;"),
     "softmax without its normalizer":
         ("u += exp(z[(size_t)r * M + i] - mx[r]) / den[r];", "u += exp(z[(size_t)r * M + i] - mx[r]);"),
+    "query heads mapped to groups interleaved":
+        ("const int h = g * G + r;\n      const int L = st->len[gi];\n      const uint16_t* qh",
+         "const int h = r * c->Hkv + g;\n      const int L = st->len[gi];\n      const uint16_t* qh"),
+    "attention output not normalised":
+        ("o[x] = (nt > 0) ? o[x] / den : 0.0;", "o[x] = (nt > 0) ? o[x] : 0.0;"),
+    "top-m takes the lowest keys":
+        ("  if (x->key > y->key) return -1;\n  if (x->key < y->key) return 1;",
+         "  if (x->key < y->key) return -1;\n  if (x->key > y->key) return 1;"),
+    "query-aware set of fixed size k_q":
+        ("const int mq = (k - ne < N - ne) ? k - ne : N - ne;", "const int mq = (c->k_q < N - ne) ? c->k_q : N - ne;"),
+    "S(t) records only Gamma_q":
+        ("ps[j] = (uint8_t)(ge[j] || gq[j]);", "ps[j] = (uint8_t)(gq[j]);"),
+    "eviction candidates ignore S(t-1)":
+        ("cand[j] = (uint8_t)(j < N && ps[j] && al[j]);", "cand[j] = (uint8_t)(j < N && al[j]);"),
+    "last_used never refreshed":
+        ("if (need[j]) lu[j] = L;", "if (need[j]) lu[j] = lu[j];"),
+    "victims paired in least-recently-used order":
+        ("for (int j = 0; j < nb; ++j)\n          if (isv[j]) vict[w++] = j;", "for (int r = 0; r < nv; ++r) vict[w++] = vc[r].idx;"),
+    "free slots taken from the top":
+        ("for (int z = 0; z < c->slots && nz < nm; ++z)\n      if (own[z] < 0) zl[nz++] = z;",
+         "for (int z = c->slots - 1; z >= 0 && nz < nm; --z)\n      if (own[z] < 0) zl[nz++] = z;"),
+    "tail block always counted a miss":
+        ("if (need[j] && bsl[j] < 0) misses[nm++] = j;", "if (need[j] && (bsl[j] < 0 || j == tail)) misses[nm++] = j;"),
+    "append refreshes the previous sub-block":
+        ("const int i = pos / c->s;\n    sub_mean", "const int i = (pos > 0 ? pos - 1 : 0) / c->s;\n    sub_mean"),
+    "sub-block assigned to the next block":
+        ("const int j = i / spb;\n      if (u > out[j])", "const int j = (i + 1) / spb;\n      if (j < nb && u > out[j])"),
+    "softmax exponent without the row max":
+        ("for (int i = 0; i < M; ++i) den[r] += exp(zr[i] - mx[r]);", "for (int i = 0; i < M; ++i) den[r] += exp(zr[i]);"),
+    "early stop without rescaling the accumulator":
+        ("for (int x = 0; x < d; ++x) acc[x] *= rescale;", "for (int x = 0; x < d; ++x) acc[x] *= 1.0;"),
+    "early stop normalises without the stopping block's mass":
+        ("if (ratio < tau_stop) break;", "if (ratio < tau_stop) { l -= dl; break; }"),
+    "window counts the next sub-block in full":
+        ("if (win && i + 1 < M) n1 = (L - (i + 1) * c->s < c->s) ? L - (i + 1) * c->s : c->s;",
+         "if (win && i + 1 < M) n1 = c->s;"),
+    "eviction set ranked by block scores":
+        ("ekey[j] = (double)evict[(size_t)gi * nb + j];", "ekey[j] = scores[(size_t)gi * nb + j];"),
+    "scale applied twice in scores":
+        ("z[(size_t)r * M + i] = c->scale * dot;", "z[(size_t)r * M + i] = c->scale * c->scale * dot;"),
+    "last prefill block starts outside S(-1)":
+        ("st->prev_sel[(size_t)gi * nb + j] = (uint8_t)(j < n0);", "st->prev_sel[(size_t)gi * nb + j] = (uint8_t)(j < n0 - 1);"),
 }
 
 

@@ -35,8 +35,9 @@ def test_hand_worked_dual_selection():
     P.check_hand_dual_selection()
 
 
-def test_hand_worked_residency():
-    P.check_hand_residency()
+@pytest.mark.parametrize("golden", ["hand_residency.json", "hand_residency_order.json"])
+def test_hand_worked_residency(golden):
+    P.check_hand_residency(name=golden)
 
 
 def test_static_eviction_closed_form():
@@ -53,7 +54,7 @@ def test_pooling_equals_library_pools(name):
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "ragged_offload", "offload_small", "sink_small", "g8",
-                                  "empty", "tiny_forecast"])
+                                  "empty", "tiny_forecast", "short_kq0", "short_kq0_offload"])
 def test_attention_and_selection_trace(name):
     case = P.check_attention_subset(CS[name])
     P.check_selection_trace(case)
