@@ -333,6 +333,25 @@ def run_gpu(args, cfg):
     def do_step(t, events=None):
         cache.step(d_q[t], d_kn[t], d_vn[t], d_ev[t], sel, out, miss_all[t, :NG], stream=stream, events=events)
 
+    # graph launch: the step is captured once (after step 0 has loaded its kernels) and
+    # replayed; each step's inputs are first copied into the graph's input buffers and its
+    # miss counts copied out afterwards, both outside the timed region
+    sg = None
+
+    def stage(t):
+        if sg is not None:
+            sg.stage(d_q[t], d_kn[t], d_vn[t], d_ev[t])
+
+    def launch(t):
+        if sg is not None:
+            sg.replay()
+        else:
+            do_step(t)
+
+    def collect(t):
+        if sg is not None:
+            miss_all[t, :NG].copy_(sg.miss[:NG])
+
     t = 0
     # step 0 (S(-1) = every prefill block; with offload, the initial residency misses) is the
     # first warm-up step, timed on its own
@@ -342,8 +361,22 @@ def run_gpu(args, cfg):
     do_step(t)
     e0_.record(stream)
     t += 1
+    torch.cuda.synchronize()
+    launch_note = "direct launches"
+    if args.launch == "graph":
+        from kv_cache_offload_nosa_b200.graph import StepGraph
+        try:
+            sg = StepGraph(cache)
+            launch_note = ("cuda graph: one captured nosa_step replayed per step, inputs staged "
+                           "into its buffers before the timed region")
+        except Exception as e:  # capture refused: time the same kernels launched directly
+            sg = None
+            launch_note = f"direct launches (graph capture failed: {type(e).__name__}: {str(e)[:120]})"
+            torch.cuda.synchronize()
     for _ in range(args.warmup - 1):
-        do_step(t)
+        stage(t)
+        launch(t)
+        collect(t)
         t += 1
     torch.cuda.synchronize()
     step0_ms = s0.elapsed_time(e0_)
@@ -359,14 +392,18 @@ def run_gpu(args, cfg):
     with Clocks(local) as clk:
         # the clock sampler's start leaves the GPU idle for a moment: one more untimed step
         # brings the clocks back up before the timed ones
+        stage(t)
         flush.zero_()
-        do_step(t)
+        launch(t)
+        collect(t)
         t += 1
         for i in range(args.steps):
+            stage(t)
             flush.zero_()
             starts[i].record(stream)
-            do_step(t)
+            launch(t)
             ends[i].record(stream)
+            collect(t)
             Ls.append((cfg.T[0] + t + 1, t))
             t += 1
         torch.cuda.synchronize()
@@ -424,6 +461,22 @@ def run_gpu(args, cfg):
                 buf[o_offs[2]:o_offs[2] + o_sizes[2]].view(torch.int32))
     views_in = [in_views(b) for b in dev_in]      # built once, outside the timed region
     views_out = [out_views(b) for b in dev_out]
+
+    def e2e_step(k):
+        bq, bk, bv, be = views_in[k]
+        o_dev, s_dev, m_dev = views_out[k]
+        cache.step(bq, bk, bv, be, s_dev, o_dev, m_dev, stream=torch.cuda.current_stream())
+
+    e2e_graphs = None
+    if sg is not None:
+        # one captured step per buffer set (capture records the launches, nothing runs)
+        e2e_graphs = []
+        for k in range(2):
+            g = torch.cuda.CUDAGraph()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, capture_error_mode="relaxed"):
+                e2e_step(k)
+            e2e_graphs.append(g)
     h2d_done = [torch.cuda.Event() for _ in range(2)]
     step_done = [torch.cuda.Event() for _ in range(2)]
     d2h_done = [torch.cuda.Event() for _ in range(2)]
@@ -447,9 +500,10 @@ def run_gpu(args, cfg):
         stream.wait_event(h2d_done[k])
         if i >= 2:
             stream.wait_event(d2h_done[k])  # step i-2's outputs have left buffer set k
-        bq, bk, bv, be = views_in[k]
-        o_dev, s_dev, m_dev = views_out[k]
-        cache.step(bq, bk, bv, be, s_dev, o_dev, m_dev, stream=stream)
+        if e2e_graphs is not None:
+            e2e_graphs[k].replay()
+        else:
+            e2e_step(k)
         step_done[k].record(stream)
         with torch.cuda.stream(ds):
             ds.wait_event(step_done[k])
@@ -521,6 +575,8 @@ def run_gpu(args, cfg):
                    "parallelism": f"replicas x{world} (batch-sharded, no collective)",
                    "l2": "flushed before every timed step (256 MiB write, then 256 MiB read so no dirty line is written back inside the timed region)",
                    "queries_per_step": q_per_step},
+        "launch": launch_note,
+        "tokens_per_s": cfg.B * world * args.steps / (tot_ms / 1e3),
         "step_us": 1e3 * tot_ms / args.steps,
         "step_us_median": 1e3 * float(np.median(step_ms)),
         "step_us_pct": {f"p{q}": 1e3 * float(np.percentile(step_ms, q)) for q in (0, 10, 50, 90, 100)},
@@ -689,6 +745,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=4, help="layers of the lookahead workload")
+    ap.add_argument("--launch", default="graph", choices=["graph", "direct"],
+                    help="timed steps as one replayed CUDA graph per step, or direct launches")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

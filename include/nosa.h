@@ -251,9 +251,9 @@ nosa_status nosa_attend(const nosa_config* cfg, const nosa_state* st, const uint
 
 /*
  * No-allocation variant of nosa_decode_attn (the pages have no counterpart: this is an
- * integration aid). Some callers cannot call cudaMalloc when they run attention: code being
- * captured into a CUDA graph, plugins inside a host framework that owns all device memory,
- * or a latency-bound serving loop that must not allocate or synchronise. This entry point
+ * integration aid). Some callers cannot call cudaMalloc when they run attention: plugins
+ * inside a host framework that owns all device memory, or a latency-bound serving loop that
+ * must not allocate or synchronise. This entry point
  * computes exactly what nosa_decode_attn computes but takes no workspace: its scratch (the
  * split-K partials and the per-group counters) lives in a static device array of 8 MiB
  * inside the library, which every GPU that loads the library keeps until the process exits.

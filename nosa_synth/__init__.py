@@ -220,8 +220,8 @@ def configs() -> dict:
     # block boundary: Gamma_e falls short while new blocks appear, and the query-aware set
     # fills S(t) up to k
     c["short_kq0"] = NosaConfig("short_kq0", 2, 8, 2, 64, (64, 96), 32, 16, 0, 5, 120, cfg_id=56)
-    c["short_kq0_offload"] = c["short_kq0"].with_(name="short_kq0_offload", slots=8, drift=0.05,
-                                                  cfg_id=57)
+    c["short_kq0_offload"] = c["short_kq0"].with_(name="short_kq0_offload", steps=250, slots=8,
+                                                  drift=0.05, cfg_id=57)
     # lookahead (SparDA order: select from the forecast row, then append, then attend)
     c["lookahead"] = c["offload"].with_(name="lookahead", n_score_rows=1, cfg_id=61)
     c["lookahead_small"] = c["offload_small"].with_(name="lookahead_small", n_score_rows=1,

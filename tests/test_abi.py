@@ -90,3 +90,17 @@ def test_status_strings(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(ImportError):
         nosa.load(str(tmp_path / "libnosa.so"))
+
+
+def test_every_synthetic_config_passes_the_library_checks(lib):
+    """Each workload the tests and the benchmark run is one the library accepts (its config
+    checks run on the host), and offload ones have the slots the state check asks for."""
+    import nosa_synth as syn
+    for name, c in syn.configs().items():
+        cc = nosa.make_config(c.B, c.Hq, c.Hkv, c.d, c.block, c.sub_block, c.k_q, c.k_e, c.max_blocks,
+                              slots=c.n_slots, n_score_rows=c.rows, scale=c.scale,
+                              score_mode=c.score_mode, stop_tau=c.stop_tau, kc_bf16=c.kc_bf16)
+        nosa.state_sizes(cc)
+        assert nosa.workspace_size(cc) > 0, name
+        if c.offload:
+            assert c.k + 2 <= c.n_slots <= c.max_blocks, (name, c.k, c.n_slots, c.max_blocks)

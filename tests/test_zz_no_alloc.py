@@ -1,8 +1,8 @@
 """nosa_decode_attn_noalloc: the workspace-free attention entry point (needs a B200).
 
-Callers that cannot allocate device memory when attention runs (graph capture,
-plugins whose host framework owns all device memory, serving loops that must
-not allocate) use this entry point; its scratch lives in a static device array
+Callers that cannot allocate device memory when attention runs (plugins whose
+host framework owns all device memory, serving loops that must not allocate)
+use this entry point; its scratch lives in a static device array
 inside the library. It must give the same output as nosa_decode_attn, call
 after call, since every call reuses (and must re-zero) the same scratch.
 
