@@ -9,6 +9,12 @@ memory, pinned host memory and streams.
 The function names mirror the C ABI of ``include/nosa.h``; tensors are passed
 by their data pointers and must already have the documented dtype, shape and
 placement.
+
+What the step computes follows NOSA: Native and Offloadable Sparse Attention
+(technical summary at gist.science/es/paper/2510.13602, "Metodologia" 1 and 2);
+the lookahead calls (plan_ahead, prefetch, attend) follow SparDA's decoupled
+selection (gist.science/de/paper/2606.04511, section 2) and the early stop
+follows S2O's stopping rule (gist.science/it/paper/2602.22575).
 """
 from __future__ import annotations
 

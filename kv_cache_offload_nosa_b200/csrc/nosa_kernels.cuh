@@ -1,5 +1,12 @@
 // Score / append / select / gather / init kernels of the NOSA decode step.
 //
+// NOSA: Native and Offloadable Sparse Attention (technical summary at
+// gist.science/es/paper/2510.13602): "Metodologia" 1, "Implementacion Basada en Bloques"
+// (each sub-block is represented by its mean key; a block's score is the max over its
+// sub-blocks' scores) and 2, "Layout de Memoria
+// Optimizado" (KV kept in minimal block units; set differences decide the pages to swap)
+// and "Comunicacion de Alto Ancho de Banda" (UVA copy kernels for the host -> HBM pages).
+//
 // score_kernel streams the fp32 sub-block mean keys (kc) of every group once:
 // HBM-bound at one FMA per 4 bytes, so it is written for coalesced 16-byte
 // loads (each warp covers whole sub-blocks with 128-byte segments), a grid of
