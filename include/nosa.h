@@ -13,8 +13,18 @@
  * Forecast-Indexer") supplies the one-forecast-row scoring variant.
  *
  * Conventions (every entry point):
- *  - Returns nosa_status; never aborts, throws or prints. A failed call
- *    launches nothing. nosa_last_error() gives a one-line reason (thread-local).
+ *  - Returns nosa_status; never aborts, throws or prints. A call refused for its
+ *    arguments (NOSA_EINVAL, NOSA_ENOMEM) launches nothing: every check comes
+ *    before the first launch. NOSA_ECUDA reports a CUDA error, which may come
+ *    after some of the call's kernels were launched. nosa_last_error() gives a
+ *    one-line reason (thread-local).
+ *  - Runs on the calling thread's current device: pointers and the stream must
+ *    belong to it (the library reads that device's SM count and sets its kernel
+ *    attributes there).
+ *  - Calls on different states and workspaces may run concurrently on any
+ *    streams. Calls that share a state or a workspace must be ordered (one
+ *    stream, or events): the kernels keep per-group flags, tickets and counters
+ *    in the workspace and update the state in place.
  *  - Asynchronous on the caller's stream (`stream` is a cudaStream_t; NULL =
  *    legacy default stream). Nothing synchronises except nosa_check_device.
  *  - The caller owns all memory: device buffers (any allocator) and, for
