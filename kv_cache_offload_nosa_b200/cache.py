@@ -11,7 +11,7 @@ import torch
 
 from . import (nosa_config, nosa_state, STATE_FIELDS, state_sizes, workspace_size, workspace_init,
                state_init, append, score_blocks, select, gather, decode_attn, step, check_device,
-               plan_ahead, prefetch, attend, stop_counts)
+               plan_ahead, prefetch, attend, stop_counts, NosaError, NOSA_EINVAL)
 
 _DTYPE = {"seq_len": torch.int32, "kc": torch.float32, "prev_sel": torch.int32,
           "alive": torch.int32, "last_used": torch.int32, "block_table": torch.int32,
@@ -19,11 +19,40 @@ _DTYPE = {"seq_len": torch.int32, "kc": torch.float32, "prev_sel": torch.int32,
           "host_k": torch.int16, "host_v": torch.int16, "err": torch.int32}
 
 
+def buffer_bytes(cfg: nosa_config) -> dict:
+    """Bytes of each per-call buffer in the layouts include/nosa.h documents."""
+    ng = cfg.B * cfg.Hkv
+    k = cfg.k_q + cfg.k_e
+    return {"q": cfg.B * cfg.Hq * cfg.d * 2, "out": cfg.B * cfg.Hq * cfg.d * 4,
+            "k_new": ng * cfg.d * 2, "v_new": ng * cfg.d * 2,
+            "score_rows": ng * cfg.n_score_rows * cfg.d * 2,
+            "block_scores": ng * cfg.max_blocks * 4, "evict": ng * cfg.max_blocks * 4,
+            "sel": ng * k * 4, "miss_count": ng * 4, "used": cfg.B * cfg.Hq * 4,
+            "prefill_len": cfg.B * 4, "resident": ng * cfg.max_blocks}
+
+
+def check_buffer(name: str, t, nbytes: int):
+    """Refuses (NosaError, NOSA_EINVAL) a tensor that is not a contiguous CUDA tensor of at
+    least `nbytes` bytes: the kernels read and write the documented extent through its data
+    pointer. Integer addresses pass unchecked, as at the C ABI."""
+    if t is None or isinstance(t, int):
+        return
+    if not t.is_cuda:
+        raise NosaError(NOSA_EINVAL, f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise NosaError(NOSA_EINVAL, f"{name} must be contiguous")
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise NosaError(NOSA_EINVAL, f"{name} holds {have} bytes, the call needs {nbytes}")
+
+
 class NosaCache:
     """Decode state + workspace for one configuration.
 
     offload=True keeps the full K/V backing copy in pinned host memory and
     `cfg.slots` pages per group in HBM; otherwise every block is in HBM.
+    Every call checks the sizes of the buffers it is given (check_buffer) before
+    the library launches anything.
     """
 
     def __init__(self, cfg: nosa_config, offload: bool = False, device: str = "cuda"):
@@ -45,6 +74,11 @@ class NosaCache:
         workspace_init(self.ws, self.ws_bytes)
         self.state = nosa_state(*[(self.t[n].data_ptr() if self.t[n] is not None else None)
                                   for n in STATE_FIELDS])
+        self._bytes = buffer_bytes(cfg)
+
+    def _check(self, **bufs):
+        for name, t in bufs.items():
+            check_buffer(name, t, self._bytes[name])
 
     # views in the documented layouts
     def pool_view(self, name: str) -> torch.Tensor:
@@ -54,29 +88,38 @@ class NosaCache:
         return self.t[name].view(G, pages, c.block_size, c.d)
 
     def init(self, prefill_len: torch.Tensor, resident: Optional[torch.Tensor] = None, stream=None):
+        self._check(prefill_len=prefill_len, resident=resident)
         state_init(self.cfg, self.state, prefill_len, resident, self.ws, self.ws_bytes, stream)
 
     def append(self, k_new, v_new, stream=None):
+        self._check(k_new=k_new, v_new=v_new)
         append(self.cfg, self.state, k_new, v_new, stream)
 
     def score_blocks(self, rows, block_scores, stream=None):
+        self._check(score_rows=rows, block_scores=block_scores)
         score_blocks(self.cfg, self.state, rows, block_scores, stream)
 
     def select(self, block_scores, evict, sel, stream=None):
+        self._check(block_scores=block_scores, evict=evict, sel=sel)
         select(self.cfg, self.state, block_scores, evict, sel, stream)
 
     def gather(self, sel, miss_count, stream=None):
+        self._check(sel=sel, miss_count=miss_count)
         gather(self.cfg, self.state, sel, miss_count, self.ws, self.ws_bytes, stream)
 
     def decode_attn(self, q, sel, out, stream=None):
+        self._check(q=q, sel=sel, out=out)
         decode_attn(self.cfg, self.state, q, sel, out, self.ws, self.ws_bytes, stream)
 
     def step(self, q, k_new, v_new, evict, sel, out, miss_count, score_rows=None, stream=None,
              events=None):
+        self._check(q=q, k_new=k_new, v_new=v_new, evict=evict, sel=sel, out=out,
+                    miss_count=miss_count, score_rows=score_rows)
         step(self.cfg, self.state, q, score_rows, k_new, v_new, evict, sel, out, miss_count, self.ws,
              self.ws_bytes, stream, events)
 
     def plan_ahead(self, score_rows, evict, sel, miss_count, stream=None):
+        self._check(score_rows=score_rows, evict=evict, sel=sel, miss_count=miss_count)
         plan_ahead(self.cfg, self.state, score_rows, evict, sel, miss_count, self.ws, self.ws_bytes,
                    stream)
 
@@ -84,9 +127,11 @@ class NosaCache:
         prefetch(self.cfg, self.state, self.ws, self.ws_bytes, stream)
 
     def attend(self, q, k_new, v_new, sel, out, stream=None):
+        self._check(q=q, k_new=k_new, v_new=v_new, sel=sel, out=out)
         attend(self.cfg, self.state, q, k_new, v_new, sel, out, self.ws, self.ws_bytes, stream)
 
     def stop_counts(self, used, stream=None):
+        self._check(used=used)
         stop_counts(self.cfg, self.ws, self.ws_bytes, used, stream)
 
     def check(self, stream=None):

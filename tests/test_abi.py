@@ -104,3 +104,63 @@ def test_every_synthetic_config_passes_the_library_checks(lib):
         assert nosa.workspace_size(cc) > 0, name
         if c.offload:
             assert c.k + 2 <= c.n_slots <= c.max_blocks, (name, c.k, c.n_slots, c.max_blocks)
+
+
+class _AsCuda:
+    """A CPU tensor that reports itself as a CUDA tensor (size checks only; nothing launches)."""
+
+    def __init__(self, t):
+        self.t = t
+        self.is_cuda = True
+
+    def is_contiguous(self):
+        return self.t.is_contiguous()
+
+    def numel(self):
+        return self.t.numel()
+
+    def element_size(self):
+        return self.t.element_size()
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_forecast", "offload_small", "ragged_offload", "g8",
+                                  "empty", "lookahead_tiny", "tiny_stop", "short_kq0"])
+def test_cache_buffer_checks_accept_the_harness_buffers(name):
+    """The NosaCache size checks accept every buffer the GPU tests pass, built the same way
+    (the oracle's records and the synthetic inputs, viewed as the library's dtypes)."""
+    import numpy as np
+    import torch
+    import nosa_synth as syn
+    import oracle as O
+    from kv_cache_offload_nosa_b200.cache import NosaCache, buffer_bytes
+    cfg = syn.configs()[name]
+    case = O.run_case(cfg, steps=2, lookahead=name.startswith("lookahead"))
+    cc = nosa.make_config(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.block, cfg.sub_block, cfg.k_q, cfg.k_e,
+                          cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows, scale=cfg.scale,
+                          score_mode=cfg.score_mode, stop_tau=cfg.stop_tau, kc_bf16=cfg.kc_bf16)
+    cache = NosaCache.__new__(NosaCache)
+    cache._bytes = buffer_bytes(cc)
+
+    def dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return _AsCuda(t.view(torch.int16) if t.dtype == torch.uint16 else t)
+
+    NG = cfg.B * cfg.Hkv
+    sel = _AsCuda(torch.empty(NG * cfg.k, dtype=torch.int32))
+    out = _AsCuda(torch.empty(cfg.B * cfg.Hq * cfg.d, dtype=torch.float32))
+    miss = _AsCuda(torch.empty(NG, dtype=torch.int32))
+    scores = _AsCuda(torch.empty(NG * cfg.max_blocks, dtype=torch.float32))
+    inp, rec = case.inputs, case.steps[0]
+    cache._check(prefill_len=dev(np.array(cfg.T, np.int32)),
+                 resident=dev(inp.resident.reshape(NG, cfg.max_blocks)) if cfg.offload else None)
+    cache._check(q=dev(rec.q), k_new=dev(inp.k_new[0]), v_new=dev(inp.v_new[0]),
+                 evict=dev(inp.evict[0]), sel=sel, out=out, miss_count=miss,
+                 score_rows=dev(rec.rows), block_scores=scores,
+                 used=_AsCuda(torch.empty(cfg.B * cfg.Hq, dtype=torch.int32)))
+    # too small, not on the device, not contiguous: refused before anything launches
+    with pytest.raises(nosa.NosaError):
+        cache._check(sel=_AsCuda(torch.empty(NG * cfg.k - 1, dtype=torch.int32)))
+    with pytest.raises(nosa.NosaError):
+        cache._check(out=torch.empty(cfg.B * cfg.Hq * cfg.d, dtype=torch.float32))
+    with pytest.raises(nosa.NosaError):
+        cache._check(q=_AsCuda(torch.empty(2 * cfg.B * cfg.Hq * cfg.d, dtype=torch.int16)[::2]))
