@@ -110,3 +110,20 @@ def test_traffic_record_needs_the_captured_source(tmp_path, monkeypatch):
     with open(csrc / "nosa_attn.cuh", "a") as f:
         f.write("// changed\n")
     assert bench.attn_traffic(16) is None
+
+
+def test_profile_commands_leave_clocks_alone_and_run_committed_files():
+    """Every ncu command recorded under profiles/ unlocks nothing it did not lock
+    (--clock-control none) and runs only the committed benchmark."""
+    import re
+    pdir = os.path.join(bench.ROOT, "profiles")
+    names = sorted(f for f in os.listdir(pdir) if f.endswith((".md", ".txt")))
+    assert names
+    for f in names:
+        text = open(os.path.join(pdir, f)).read()
+        cmds = [l for l in text.splitlines() if re.search(r"(^|\s)ncu\s+--", l)]
+        assert cmds, f"{f}: no ncu command recorded"
+        for l in cmds:
+            assert "--clock-control none" in l, (f, l)
+        for script in re.findall(r"python\s+(\S+\.py)", text):
+            assert os.path.exists(os.path.join(bench.ROOT, script)), (f, script)
