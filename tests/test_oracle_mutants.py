@@ -106,3 +106,75 @@ def test_pins_catch_mutant(name, tmp_path):
     so = O.compile_oracle(str(path), str(tmp_path / f"libm_{abs(hash(name))}.so"))
     with pytest.raises((AssertionError, RuntimeError, ValueError)):
         P.run_all(so)
+
+
+# Slips in the oracle's Python driver (the SparDA lookahead order of run_case). Each runs the
+# lookahead pins in a child process on a copy of the oracle package with one change.
+PY_MUTANTS = {
+    "lookahead appends before selecting":
+        [("        if not lookahead:\n            orc.append(inp.k_new[t], inp.v_new[t])",
+          "        if True:\n            orc.append(inp.k_new[t], inp.v_new[t])"),
+         ("        if lookahead:\n            orc.append(inp.k_new[t], inp.v_new[t])",
+          "        if False:\n            orc.append(inp.k_new[t], inp.v_new[t])")],
+    "lookahead plans residency after the append":
+        [("        miss = orc.residency(sel)\n        if lookahead:\n            orc.append(inp.k_new[t], inp.v_new[t])",
+          "        if lookahead:\n            orc.append(inp.k_new[t], inp.v_new[t])\n        miss = orc.residency(sel)")],
+    "lookahead attends before the append":
+        [("        if lookahead:\n            orc.append(inp.k_new[t], inp.v_new[t])\n        used = None",
+          "        used = None"),
+         ("            out = orc.attend(q16, sel)\n",
+          "            out = orc.attend(q16, sel)\n            if lookahead:\n                orc.append(inp.k_new[t], inp.v_new[t])\n")],
+}
+
+_PY_DRIVER = """
+import sys
+sys.path.insert(0, {pkg!r})
+sys.path.insert(1, {root!r})
+sys.path.insert(2, {tests!r})
+import oracle as O
+assert O.__file__.startswith({pkg!r}), O.__file__
+import nosa_synth as syn
+import oracle_pins as P
+P.check_lookahead_dense_sdpa()
+cs = syn.configs()
+for name in ("lookahead_tiny", "lookahead_ragged", "lookahead_small"):
+    case = P.check_attention_subset(cs[name], lookahead=True)
+    P.check_selection_trace(case, lookahead=True)
+    if case.cfg.offload:
+        P.check_residency_trace(case, lookahead=True)
+print("LOOKAHEAD PINS PASS")
+"""
+
+
+def _run_py_mutant(tmp_path, edits):
+    import shutil
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = tmp_path / "pkg"
+    dst = pkg / "oracle"
+    dst.mkdir(parents=True)
+    src_dir = os.path.join(root, "oracle")
+    for f in ("__init__.py", "nosa_oracle.c"):
+        shutil.copy(os.path.join(src_dir, f), dst / f)
+    shutil.copy(O.build(), dst / "libnosa_oracle.so")
+    text = (dst / "__init__.py").read_text()
+    for old, new in edits:
+        assert text.count(old) == 1, f"mutation site not unique: {old[:60]!r}"
+        text = text.replace(old, new)
+    (dst / "__init__.py").write_text(text)
+    drv = tmp_path / "drive.py"
+    drv.write_text(_PY_DRIVER.format(pkg=str(pkg), root=root, tests=os.path.join(root, "tests")))
+    return subprocess.run([sys.executable, str(drv)], capture_output=True, text=True, timeout=900)
+
+
+def test_lookahead_pins_pass_on_the_unchanged_driver(tmp_path):
+    r = _run_py_mutant(tmp_path, [])
+    assert r.returncode == 0 and "LOOKAHEAD PINS PASS" in r.stdout, r.stderr[-3000:]
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_lookahead_pins_catch_driver_mutant(name, tmp_path):
+    r = _run_py_mutant(tmp_path, PY_MUTANTS[name])
+    assert r.returncode != 0 and "LOOKAHEAD PINS PASS" not in r.stdout, r.stdout[-2000:]
+    assert "AssertionError" in r.stderr or "ValueError" in r.stderr, r.stderr[-3000:]
