@@ -99,6 +99,10 @@ typedef struct nosa_config {
   int32_t kc_bf16;        /* 1: state->kc holds bf16 sub-block means (each mean is summed in fp32 in
                              token order, divided in fp32 and rounded to nearest even), half the
                              score kernel's bytes; 0: fp32 means. */
+  int32_t wait_us;        /* limit of every bounded device wait (a per-group flag, an mbarrier), in
+                             microseconds from the waiting kernel's start, in [0, 60000000];
+                             0 = 4 s. A wait that runs out sets NOSA_ERR_TIMEOUT and the kernel
+                             returns; nosa_check_device then reports NOSA_ETIMEOUT. */
 } nosa_config;
 
 #define NOSA_SCORE_WINDOW 1

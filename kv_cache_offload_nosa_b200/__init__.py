@@ -43,7 +43,8 @@ class nosa_config(ctypes.Structure):
                  "slots", "n_score_rows", "attn_split")] + [("scale", ctypes.c_float),
                                                              ("score_mode", ctypes.c_int32),
                                                              ("stop_tau", ctypes.c_float),
-                                                             ("kc_bf16", ctypes.c_int32)]
+                                                             ("kc_bf16", ctypes.c_int32),
+                                                             ("wait_us", ctypes.c_int32)]
 
 
 STATE_FIELDS = ("seq_len", "kc", "prev_sel", "alive", "last_used", "block_table", "slot_owner",
@@ -135,12 +136,12 @@ def _stream(stream) -> Optional[int]:
 
 def make_config(B, Hq, Hkv, d, block_size, sub_block, k_q, k_e, max_blocks, slots=None,
                 n_score_rows=None, attn_split=0, scale=None, score_mode=0, stop_tau=0.0,
-                kc_bf16=0) -> nosa_config:
+                kc_bf16=0, wait_us=0) -> nosa_config:
     G = Hq // Hkv
     return nosa_config(B, Hq, Hkv, d, block_size, sub_block, k_q, k_e, max_blocks,
                        max_blocks if slots is None else slots, G if n_score_rows is None else n_score_rows,
                        attn_split, (1.0 / d ** 0.5) if scale is None else scale, score_mode, stop_tau,
-                       kc_bf16)
+                       kc_bf16, wait_us)
 
 
 def state_sizes(cfg: nosa_config) -> nosa_sizes:

@@ -31,14 +31,18 @@ def buffer_bytes(cfg: nosa_config) -> dict:
             "prefill_len": cfg.B * 4, "resident": ng * cfg.max_blocks}
 
 
-def check_buffer(name: str, t, nbytes: int):
+def check_buffer(name: str, t, nbytes: int, device: Optional[torch.device] = None):
     """Refuses (NosaError, NOSA_EINVAL) a tensor that is not a contiguous CUDA tensor of at
-    least `nbytes` bytes: the kernels read and write the documented extent through its data
-    pointer. Integer addresses pass unchecked, as at the C ABI."""
+    least `nbytes` bytes on `device` (the GPU that holds the state): the kernels read and write
+    the documented extent through its data pointer, and a pointer into another GPU's memory
+    would fault there instead of failing here. Integer addresses pass unchecked, as at the C
+    ABI."""
     if t is None or isinstance(t, int):
         return
     if not t.is_cuda:
         raise NosaError(NOSA_EINVAL, f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise NosaError(NOSA_EINVAL, f"{name} is on {t.device}, the state is on {device}")
     if not t.is_contiguous():
         raise NosaError(NOSA_EINVAL, f"{name} must be contiguous")
     have = t.numel() * t.element_size()
@@ -69,6 +73,8 @@ class NosaCache:
                 self.t[name] = (torch.empty(n, dtype=dt, pin_memory=True) if offload else None)
             else:
                 self.t[name] = torch.empty(n, dtype=dt, device=self.device)
+        # the state's own device, with its index (the buffers of every call must be there)
+        self.device = self.t["seq_len"].device
         self.ws_bytes = workspace_size(cfg)
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
         workspace_init(self.ws, self.ws_bytes)
@@ -78,7 +84,7 @@ class NosaCache:
 
     def _check(self, **bufs):
         for name, t in bufs.items():
-            check_buffer(name, t, self._bytes[name])
+            check_buffer(name, t, self._bytes[name], self.device)
 
     # views in the documented layouts
     def pool_view(self, name: str) -> torch.Tensor:

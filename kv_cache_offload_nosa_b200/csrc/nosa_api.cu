@@ -73,6 +73,7 @@ nosa_status check_cfg(const nosa_config* cp) {
   NOSA_CHECK(c.kc_bf16 == 0 || c.kc_bf16 == 1, "kc_bf16 must be 0 or 1");
   NOSA_CHECK(!(c.stop_tau > 0.f) || kk(c) <= kStopMaxK, "early stop supports k <= %d", kStopMaxK);
   NOSA_CHECK(c.scale > 0.f, "scale must be > 0");
+  NOSA_CHECK(c.wait_us >= 0 && c.wait_us <= 60000000, "wait_us = %d not in [0, 60000000]", c.wait_us);
   const long long groups = (long long)c.B * c.Hkv;
   NOSA_CHECK(groups * c.slots * c.block_size < (1ll << 31), "too many pool rows for TMA coordinates");
   NOSA_CHECK(groups * kk(c) < (1ll << 31), "too many tasks");
@@ -80,6 +81,11 @@ nosa_status check_cfg(const nosa_config* cp) {
 }
 
 bool has_host(const nosa_state* st) { return st->host_k != nullptr; }
+
+// Limit of the kernels' bounded waits, in ns.
+unsigned long long wait_ns(const nosa_config& c) {
+  return c.wait_us > 0 ? (unsigned long long)c.wait_us * 1000ull : kWaitLimitNs;
+}
 
 nosa_status check_state(const nosa_config& c, const nosa_state* st) {
   NOSA_CHECK(st, "state is NULL");
@@ -180,6 +186,7 @@ StepArgs step_args(const nosa_config& c, const nosa_state* st) {
   a.slot_owner = st->slot_owner;
   a.last_used = st->last_used;
   a.err = st->err;
+  a.wait_ns = wait_ns(c);
   return a;
 }
 
@@ -252,6 +259,7 @@ nosa_status launch_copy(const nosa_config& c, const nosa_state* st, void* ws, cu
   ca.copy_cnt = ws_at<uint32_t>(ws, w.copy_cnt);
   ca.copy_flag = ws_at<uint32_t>(ws, w.copy_flag);
   ca.err = st->err;
+  ca.wait_ns = wait_ns(c);
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(n_groups(c), 8);
   lc.blockDim = dim3(256);
@@ -389,17 +397,10 @@ nosa_status launch_attn_stop_t(const nosa_config& c, AttnArgs a, StopArgs x, con
   return NOSA_OK;
 }
 
-// ready: per-group flags the attention waits on (and clears), or NULL to wait for the
-// previous grid as a whole. pdl: may start while the previous kernel on the stream runs.
-nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16_t* q, const int32_t* sel,
-                        float* out, void* ws, cudaStream_t s, uint32_t* ready = nullptr,
-                        bool pdl = true) {
-  CUtensorMap tk, tv;
-  nosa_status r = make_pool_map(&tk, c, st->k_pool);
-  if (r != NOSA_OK) return r;
-  r = make_pool_map(&tv, c, st->v_pool);
-  if (r != NOSA_OK) return r;
-  const WsLayout w = ws_layout(c);
+// Arguments of the split-K attention over the state's pools. partials / counters: the
+// scratch of the split-K merge (the workspace's, or the no-allocation entry point's).
+AttnArgs attn_args(const nosa_config& c, const nosa_state* st, const uint16_t* q, const int32_t* sel,
+                   float* out, float* partials, uint32_t* counters) {
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   a.q = q;
@@ -407,8 +408,8 @@ nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16
   a.seq_len = st->seq_len;
   a.block_table = st->block_table;
   a.out = out;
-  a.partials = ws_at<float>(ws, w.partials);
-  a.counters = ws_at<uint32_t>(ws, w.cnt_attn);
+  a.partials = partials;
+  a.counters = counters;
   a.err = st->err;
   a.Hq = c.Hq;
   a.Hkv = c.Hkv;
@@ -418,8 +419,41 @@ nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16
   a.total = n_groups(c) * kk(c);
   a.total_pages = (long long)n_groups(c) * c.slots;
   a.scale_log2 = c.scale * 1.4426950408889634f;
-  a.sel_flag = ready;
   a.identity = !has_host(st);
+  a.wait_ns = wait_ns(c);
+  return a;
+}
+
+nosa_status make_pool_maps(const nosa_config& c, const nosa_state* st, CUtensorMap* tk, CUtensorMap* tv) {
+  nosa_status r = make_pool_map(tk, c, st->k_pool);
+  if (r != NOSA_OK) return r;
+  return make_pool_map(tv, c, st->v_pool);
+}
+
+// The split-K attention kernel instantiated for the configuration's head dim and block size.
+nosa_status dispatch_attn(const nosa_config& c, const AttnArgs& a, const CUtensorMap& tk,
+                          const CUtensorMap& tv, cudaStream_t s, bool finest, bool pdl) {
+  if (c.d == 128) {
+    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s, finest, pdl);
+    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s, finest, pdl);
+    return launch_attn_t<128, 128>(c, a, tk, tv, s, finest, pdl);
+  }
+  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s, finest, pdl);
+  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s, finest, pdl);
+  return launch_attn_t<64, 128>(c, a, tk, tv, s, finest, pdl);
+}
+
+// ready: per-group flags the attention waits on (and clears), or NULL to wait for the
+// previous grid as a whole. pdl: may start while the previous kernel on the stream runs.
+nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16_t* q, const int32_t* sel,
+                        float* out, void* ws, cudaStream_t s, uint32_t* ready = nullptr,
+                        bool pdl = true) {
+  CUtensorMap tk, tv;
+  nosa_status r = make_pool_maps(c, st, &tk, &tv);
+  if (r != NOSA_OK) return r;
+  const WsLayout w = ws_layout(c);
+  AttnArgs a = attn_args(c, st, q, sel, out, ws_at<float>(ws, w.partials), ws_at<uint32_t>(ws, w.cnt_attn));
+  a.sel_flag = ready;
   if (c.stop_tau > 0.f) {
     // early stop: one CTA per group, after the whole previous grid (no per-group flags)
     StopArgs x;
@@ -436,14 +470,7 @@ nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16
     return launch_attn_stop_t<64, 128>(c, a, x, tk, tv, s, pdl);
   }
   const bool finest = ready != nullptr && has_host(st);
-  if (c.d == 128) {
-    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s, finest, pdl);
-    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s, finest, pdl);
-    return launch_attn_t<128, 128>(c, a, tk, tv, s, finest, pdl);
-  }
-  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s, finest, pdl);
-  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s, finest, pdl);
-  return launch_attn_t<64, 128>(c, a, tk, tv, s, finest, pdl);
+  return dispatch_attn(c, a, tk, tv, s, finest, pdl);
 }
 
 }  // namespace
@@ -822,39 +849,14 @@ extern "C" nosa_status nosa_decode_attn_noalloc(const nosa_config* cfg, const no
   void* base = nullptr;
   if ((r = noalloc_scratch(&base)) != NOSA_OK) return r;
   cudaStream_t s = as_stream(stream);
+  // every check (the tensor maps included) before the first work is queued on the stream
+  CUtensorMap tk, tv;
+  if ((r = make_pool_maps(c, st, &tk, &tv)) != NOSA_OK) return r;
   uint32_t* counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(base) + part_bytes);
   // the array keeps the previous call's contents: the last-arriver counters must start at zero
   NOSA_CUDA(cudaMemsetAsync(counters, 0, NG * 4, s));
-  CUtensorMap tk, tv;
-  if ((r = make_pool_map(&tk, c, st->k_pool)) != NOSA_OK) return r;
-  if ((r = make_pool_map(&tv, c, st->v_pool)) != NOSA_OK) return r;
-  AttnArgs a;
-  memset(&a, 0, sizeof(a));
-  a.q = q;
-  a.sel = sel;
-  a.seq_len = st->seq_len;
-  a.block_table = st->block_table;
-  a.out = out;
-  a.partials = static_cast<float*>(base);
-  a.counters = counters;
-  a.err = st->err;
-  a.Hq = c.Hq;
-  a.Hkv = c.Hkv;
-  a.G = c.Hq / c.Hkv;
-  a.k = kk(c);
-  a.max_blocks = c.max_blocks;
-  a.total = n_groups(c) * kk(c);
-  a.total_pages = (long long)n_groups(c) * c.slots;
-  a.scale_log2 = c.scale * 1.4426950408889634f;
-  const bool finest = false;
-  if (c.d == 128) {
-    if (c.block_size == 32) return launch_attn_t<128, 32>(c, a, tk, tv, s, finest);
-    if (c.block_size == 64) return launch_attn_t<128, 64>(c, a, tk, tv, s, finest);
-    return launch_attn_t<128, 128>(c, a, tk, tv, s, finest);
-  }
-  if (c.block_size == 32) return launch_attn_t<64, 32>(c, a, tk, tv, s, finest);
-  if (c.block_size == 64) return launch_attn_t<64, 64>(c, a, tk, tv, s, finest);
-  return launch_attn_t<64, 128>(c, a, tk, tv, s, finest);
+  const AttnArgs a = attn_args(c, st, q, sel, out, static_cast<float*>(base), counters);
+  return dispatch_attn(c, a, tk, tv, s, /*finest=*/false, /*pdl=*/true);
 }
 
 // ====================================================================== PCIe read ceiling

@@ -45,6 +45,7 @@ struct AttnArgs {
   uint32_t* sel_flag;         // [B*Hkv * kFlagStride] per-group "ready" flags, or NULL
   int identity;               // no host pools: block j of group g is page g * max_blocks + j
                               // (the state's block table is that identity), so no lookup
+  unsigned long long wait_ns; // limit of every bounded wait, from the kernel's start
 };
 
 struct TaskInfo {
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
   // either wait for that whole grid, or (flags) for the one group a task belongs to
   const bool flags = a.sel_flag != nullptr;
   if (!flags) griddep_wait();
-  const unsigned long long deadline = globaltimer() + kWaitLimitNs;
+  const unsigned long long deadline = globaltimer() + a.wait_ns;
 
   if (warp == NC) {
     // ---------------------------------------------------------------- producer

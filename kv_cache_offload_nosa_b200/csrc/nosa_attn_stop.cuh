@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
   }
   // sel, the block scores, seq_len and the block table come from the previous kernels
   griddep_wait();
-  const unsigned long long deadline = globaltimer() + kWaitLimitNs;
+  const unsigned long long deadline = globaltimer() + a.wait_ns;
   const int L = __ldcg(a.seq_len + gi);
   const int N = (L + BS - 1) / BS;
   // visiting order: selected blocks by decreasing score, ties to the lower index

@@ -17,7 +17,7 @@ constexpr int kPartialSlots = 16;          // split-K segments per group
 // Per-group flags sit 128 bytes apart (one cache line each): waiters of different groups
 // poll different lines, so no single L2 slice takes every poll.
 constexpr int kFlagStride = 32;            // uint32 words between consecutive groups' flags
-constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // bounded spin: 4 s
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // default bounded spin: 4 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -125,6 +125,13 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
+}
+// Transpose of an 8x8 b16 matrix held one 32-bit pair per lane (row lane/4, columns
+// 2*(lane%4) and 2*(lane%4) + 1) into the same layout.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
 }
 // D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate.
 // a0/a2: rows 0..7 (k 0..7 / 8..15), a1/a3: rows 8..15.

@@ -66,6 +66,7 @@ struct StepArgs {
   int kc16;               // kc holds bf16 means (else fp32)
   int mode;               // scoring variant bits (1 windows, 2 per-row softmax); 0 = NOSA pool
   float* units;           // variants: per-sub-block values [B*Hkv][rows][max_sub] (workspace)
+  unsigned long long wait_ns;  // limit of the bounded waits (append_kernel's flag)
 };
 
 constexpr int kMaxSoftRows = 8;  // scoring rows the per-row softmax variant supports
@@ -442,7 +443,7 @@ __global__ void __launch_bounds__(128) append_kernel(StepArgs a) {
   const int gi = blockIdx.x;
   if (a.ready) {
     // lookahead: this group's page copies may target the tail block; they land first
-    if (threadIdx.x == 0 && !wait_flag(a.ready + (size_t)gi * kFlagStride, globaltimer() + kWaitLimitNs))
+    if (threadIdx.x == 0 && !wait_flag(a.ready + (size_t)gi * kFlagStride, globaltimer() + a.wait_ns))
       set_err(a.err, NOSA_ERR_TIMEOUT);
     __syncthreads();
   }
@@ -511,6 +512,7 @@ struct CopyArgs {
   uint32_t* copy_cnt;    // [groups] CTAs done with the group (copy_seq_kernel; starts, ends at 0)
   uint32_t* copy_flag;   // [groups * kFlagStride] pages in place (copy_seq_kernel)
   uint32_t* err;
+  unsigned long long wait_ns;  // limit of the bounded waits on the plan flags
 };
 
 __global__ void __launch_bounds__(256) copy_kernel(CopyArgs a) {
@@ -552,7 +554,7 @@ __global__ void __launch_bounds__(256) copy_kernel(CopyArgs a) {
 __global__ void __launch_bounds__(256) copy_seq_kernel(CopyArgs a, int ngroups) {
   griddep_launch_dependents();
   __shared__ int s_n;
-  const unsigned long long deadline = globaltimer() + kWaitLimitNs;
+  const unsigned long long deadline = globaltimer() + a.wait_ns;
   for (int gi = 0; gi < ngroups; ++gi) {
     if (threadIdx.x == 0) {
       if (!wait_flag(a.sel_flag + (size_t)gi * kFlagStride, deadline)) set_err(a.err, NOSA_ERR_TIMEOUT);

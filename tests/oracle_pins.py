@@ -31,11 +31,36 @@ import oracle as O
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 
-def _tokens(case_or_orc, gi, L):
-    orc = case_or_orc
-    K = syn.bf16_to_f64(orc.K[gi // orc.cfg.Hkv, gi % orc.cfg.Hkv, :L])
-    V = syn.bf16_to_f64(orc.V[gi // orc.cfg.Hkv, gi % orc.cfg.Hkv, :L])
+_INPUTS = [None, None]  # (config key, inputs): the last configuration's fresh inputs
+
+
+def _input_tokens(cfg, gi, L):
+    """Tokens 0..L-1 of group gi as the inputs define them, drawn afresh from the generator
+    (not read from any array the oracle wrote): the prefill rows < T, then the token of
+    decode step t at position T + t (k_new[t], v_new[t]). Raw bf16 bit patterns."""
+    key = repr(cfg)
+    if _INPUTS[0] != key:
+        _INPUTS[:] = [key, syn.make_inputs(cfg)]
+    inp = _INPUTS[1]
+    b, g = gi // cfg.Hkv, gi % cfg.Hkv
+    T = cfg.T[b]
+    n = L - T
+    assert 0 <= n <= inp.k_new.shape[0], (L, T)
+    K = np.concatenate([inp.pool_k[b, g, :T], inp.k_new[:n, b, g]])
+    V = np.concatenate([inp.pool_v[b, g, :T], inp.v_new[:n, b, g]])
     return K, V
+
+
+def _tokens(orc, gi, L):
+    """Keys and values (fp64) of tokens 0..L-1 of group gi, from the inputs. The oracle's own
+    token store must hold exactly these rows: that pins its append (NOSA, "Layout de Memoria
+    Optimizado": the appended token goes to position L-1 of its group's block-unit store,
+    K from k_new and V from v_new)."""
+    K, V = _input_tokens(orc.cfg, gi, L)
+    b, g = gi // orc.cfg.Hkv, gi % orc.cfg.Hkv
+    np.testing.assert_array_equal(orc.K[b, g, :L].view(np.uint16), K, err_msg=f"K store, group {gi}")
+    np.testing.assert_array_equal(orc.V[b, g, :L].view(np.uint16), V, err_msg=f"V store, group {gi}")
+    return syn.bf16_to_f64(K), syn.bf16_to_f64(V)
 
 
 # ----------------------------------------------------------------- top-m
@@ -390,8 +415,7 @@ def check_kc_bf16(cfg, lib_path=None, steps=2):
         b, g = gi // c.Hkv, gi % c.Hkv
         Lt = c.T[b] + t + 1
         M, N = -(-Lt // s), -(-Lt // c.block)
-        Kb = orc.K[b, g, :Lt].view(np.uint16)
-        K32 = syn.bf16_to_f64(Kb).astype(np.float32)
+        K32 = _tokens(orc, gi, Lt)[0].astype(np.float32)
         want = np.empty((M, c.d), np.float64)
         for i in range(M):
             t0, t1 = i * s, min((i + 1) * s, Lt)

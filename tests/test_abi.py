@@ -46,7 +46,7 @@ def cfg(**kw):
                                  dict(k_q=30, k_e=20), dict(max_blocks=9000), dict(slots=0),
                                  dict(n_score_rows=2), dict(scale=0.0), dict(sub_block=128),
                                  dict(score_mode=4), dict(score_mode=-1), dict(kc_bf16=2),
-                                 dict(stop_tau=-1.0)])
+                                 dict(stop_tau=-1.0), dict(wait_us=-1), dict(wait_us=60000001)])
 def test_bad_config_is_rejected_on_host(lib, bad):
     c = cfg(**bad)
     n = ctypes.c_size_t()
@@ -109,9 +109,11 @@ def test_every_synthetic_config_passes_the_library_checks(lib):
 class _AsCuda:
     """A CPU tensor that reports itself as a CUDA tensor (size checks only; nothing launches)."""
 
-    def __init__(self, t):
+    def __init__(self, t, device=None):
+        import torch
         self.t = t
         self.is_cuda = True
+        self.device = device if device is not None else torch.device("cuda", 0)
 
     def is_contiguous(self):
         return self.t.is_contiguous()
@@ -140,6 +142,7 @@ def test_cache_buffer_checks_accept_the_harness_buffers(name):
                           score_mode=cfg.score_mode, stop_tau=cfg.stop_tau, kc_bf16=cfg.kc_bf16)
     cache = NosaCache.__new__(NosaCache)
     cache._bytes = buffer_bytes(cc)
+    cache.device = torch.device("cuda", 0)
 
     def dev(a):
         t = torch.from_numpy(np.ascontiguousarray(a))
@@ -164,3 +167,23 @@ def test_cache_buffer_checks_accept_the_harness_buffers(name):
         cache._check(out=torch.empty(cfg.B * cfg.Hq * cfg.d, dtype=torch.float32))
     with pytest.raises(nosa.NosaError):
         cache._check(q=_AsCuda(torch.empty(2 * cfg.B * cfg.Hq * cfg.d, dtype=torch.int16)[::2]))
+    # the right size on another GPU: refused (its pointer is not the state's device's memory)
+    with pytest.raises(nosa.NosaError, match="state is on"):
+        cache._check(sel=_AsCuda(torch.empty(NG * cfg.k, dtype=torch.int32), torch.device("cuda", 1)))
+
+
+def test_workspace_one_byte_short_is_refused_before_any_cuda_call(lib):
+    """nosa_step with a workspace one byte below nosa_workspace_size returns NOSA_ENOMEM from
+    its argument checks, before any CUDA call (the addresses are never dereferenced: no GPU
+    is needed), and the reason names both sizes."""
+    c = cfg()
+    need = nosa.workspace_size(c)
+    fake = [0x10000 * (i + 1) for i in range(12)]           # 16-byte aligned, never read
+    st = nosa.nosa_state(*fake[:9], None, None, fake[9])   # no host pools: no pointer query
+    args = [0x200000 + 0x1000 * i for i in range(7)]       # q, k_new, v_new, evict, sel, out, miss
+    q, kn, vn, ev, sel, out, miss = args
+    rc = lib.nosa_step(ctypes.byref(c), ctypes.byref(st), q, None, kn, vn, ev, sel, out, miss,
+                       0x4000000, need - 1, None, None)
+    assert rc == nosa.NOSA_ENOMEM
+    msg = lib.nosa_last_error().decode()
+    assert str(need) in msg and str(need - 1) in msg, msg

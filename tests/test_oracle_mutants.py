@@ -91,6 +91,14 @@ MUTANTS = {
         ("ekey[j] = (double)evict[(size_t)gi * nb + j];", "ekey[j] = scores[(size_t)gi * nb + j];"),
     "scale applied twice in scores":
         ("z[(size_t)r * M + i] = c->scale * dot;", "z[(size_t)r * M + i] = c->scale * c->scale * dot;"),
+    "append writes K and V one row late":
+        ("memcpy(st->K + tok_off(c, gi, pos), k_new + (size_t)gi * c->d, sizeof(uint16_t) * c->d);\n"
+         "    memcpy(st->V + tok_off(c, gi, pos), v_new",
+         "memcpy(st->K + tok_off(c, gi, pos + 1 < c->max_blocks * c->bs ? pos + 1 : pos), k_new + (size_t)gi * c->d, sizeof(uint16_t) * c->d);\n"
+         "    memcpy(st->V + tok_off(c, gi, pos + 1 < c->max_blocks * c->bs ? pos + 1 : pos), v_new"),
+    "append copies V from k_new":
+        ("memcpy(st->V + tok_off(c, gi, pos), v_new + (size_t)gi * c->d",
+         "memcpy(st->V + tok_off(c, gi, pos), k_new + (size_t)gi * c->d"),
     "last prefill block starts outside S(-1)":
         ("st->prev_sel[(size_t)gi * nb + j] = (uint8_t)(j < n0);", "st->prev_sel[(size_t)gi * nb + j] = (uint8_t)(j < n0 - 1);"),
 }

@@ -19,14 +19,21 @@ import oracle as O
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def prepared():
+# (workload, attention split): all blocks in HBM at the automatic split; host pools, so the
+# kernel reads the block table; and a split that does not divide k, so CTA ranges cross group
+# boundaries and several segments of a group share the static partials.
+CASES = [("llama_small", 0), ("offload_small", 0), ("llama_small", 7), ("offload_small", 3)]
+
+
+@pytest.fixture(scope="module", params=CASES, ids=[f"{n}-W{w}" for n, w in CASES])
+def prepared(request):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import gpu_harness as H
-    case = O.run_case(syn.configs()["llama_small"], steps=2)
+    name, split = request.param
+    case = O.run_case(syn.configs()[name], steps=2)
     cfg = case.cfg
-    cache = H.setup(cfg, case.inputs)
+    cache = H.setup(cfg, case.inputs, attn_split=split)
     io = H.StepIO(cfg)
     H.run_step(cache, cfg, case.inputs, case.steps[0], 0, io)   # a real step: append, select, attend
     q = H.dev(case.steps[0].q)
