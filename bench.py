@@ -151,25 +151,27 @@ class Clocks:
                 "reasons": sorted(reasons)}
 
 
-def attn_traffic(batch: int):
-    """DRAM bytes per attention launch from the committed ncu summary, scaled from its batch to
-    `batch` (traffic grows with the number of groups); None when the kernel source changed
-    since the capture."""
+def kernel_source_sha(root: str = None) -> str:
+    """sha256 of the attention kernel's source (the files a traffic record was captured from)."""
     import hashlib
-    import re
-    p = os.path.join(ROOT, "profiles", "attn_kernel_llama_b8.md")
-    if not os.path.exists(p):
-        return None
-    m = re.search(r"traffic-record: batch=(\d+) dram_bytes_per_launch=(\d+) source_sha256=([0-9a-f]+)",
-                  open(p).read())
-    if not m:
-        return None
     h = hashlib.sha256()
     for f in ("nosa_attn.cuh", "nosa_common.cuh"):
-        h.update(open(os.path.join(ROOT, "kv_cache_offload_nosa_b200", "csrc", f), "rb").read())
-    if h.hexdigest() != m.group(3):
+        h.update(open(os.path.join(root or ROOT, "kv_cache_offload_nosa_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def attn_traffic(batch: int):
+    """DRAM bytes per attention launch from the committed traffic record
+    (profiles/attn_traffic.json, written from one ncu capture), scaled from its batch to
+    `batch` (traffic grows with the number of groups); None when the record is missing or the
+    kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(p):
         return None
-    return int(m.group(2)) * batch / int(m.group(1))
+    rec = json.load(open(p))
+    if rec.get("source_sha256") != kernel_source_sha():
+        return None
+    return int(rec["dram_bytes_per_launch"]) * batch / int(rec["batch"])
 
 
 def peaks():
@@ -181,23 +183,31 @@ def peaks():
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_sample(cfg: syn.NosaConfig, steps: int, budget_s: float = 20.0):
+def _omp(fn: str, *a):
+    """Calls libgomp (the OpenMP runtime the oracle's parallel regions use) in this process."""
+    import ctypes
+    try:
+        return getattr(ctypes.CDLL("libgomp.so.1"), fn)(*a)
+    except (OSError, AttributeError):
+        return None
+
+
+def oracle_sample(cfg: syn.NosaConfig, steps: int, budget_s: float = 20.0, batch: int = 2,
+                  min_steps: int = 3):
     """Times the fp64 oracle (append, score, select, residency, attention) on a bounded
-    sample of the workload: the first batch entries of the same layer, `steps` decode steps."""
+    sample of the workload: the first `batch` entries of the same layer, decode steps until
+    `budget_s` of oracle time (at least `min_steps`, at most `steps`)."""
     import oracle as O
-    B_s = max(1, min(cfg.B, 2))
+    B_s = max(1, min(cfg.B, batch))
     sub = cfg.with_(name=cfg.name + "_sample", B=B_s, T=cfg.T[:B_s], steps=steps)
     inp = syn.make_inputs(sub)
     orc = O.Oracle(sub, inp.pool_k, inp.pool_v, inp.resident)
     prev = None
     zero = np.zeros((sub.B, sub.Hkv), np.int64)
-    qs_all = []
-    for t in range(steps):
-        prev = syn.query_step(sub, t, prev, zero)
-        qs_all.append(syn.round_bf16(prev))
     times = []
     for t in range(steps):
-        q16 = qs_all[t]
+        prev = syn.query_step(sub, t, prev, zero)
+        q16 = syn.round_bf16(prev)
         t0 = time.perf_counter()
         orc.append(inp.k_new[t], inp.v_new[t])
         rows = q16.reshape(sub.B, sub.Hkv, sub.G, sub.d)
@@ -206,14 +216,30 @@ def oracle_sample(cfg: syn.NosaConfig, steps: int, budget_s: float = 20.0):
         orc.residency(sel)
         orc.attend(q16, sel)
         times.append(time.perf_counter() - t0)
-        if sum(times) > budget_s:
+        if len(times) >= min_steps and sum(times) > budget_s:
             break
     n = len(times)
     tot = sum(times)
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cores = _omp("omp_get_max_threads") or int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return {"value": sub.B * sub.Hq * n / tot, "unit": "queries/s", "cores": cores, "kind": "oracle",
             "sample": f"{n} decode steps of {B_s} of {cfg.B} batch entries of the same layer "
                       f"(fp64 C oracle, OpenMP over groups), {tot:.2f} s"}, times
+
+
+def cpu_baseline(args):
+    """The oracle on this host: all cores (OpenMP over groups) for about `cpu_budget` seconds
+    of oracle time, then one thread for about a third of that."""
+    budget = min(args.cpu_budget, 3.0)
+    cfg = workload(args.workload, 400)
+    cb, _ = oracle_sample(cfg, 400, budget_s=budget, batch=4)
+    cores = cb["cores"]
+    _omp("omp_set_num_threads", 1)
+    one, _ = oracle_sample(cfg, 400, budget_s=budget / 3, batch=4, min_steps=2)
+    _omp("omp_set_num_threads", int(cores))
+    if one["cores"] == 1:  # the runtime took the one-thread setting
+        cb["one_thread"] = {"value": one["value"], "unit": one["unit"], "cores": 1,
+                            "sample": one["sample"]}
+    return cb
 
 
 def run_reference(args, cfg):
@@ -239,17 +265,13 @@ def run_reference(args, cfg):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_gpu(args, cfg):
+def measure_gpu(args, cfg, rank, world, local):
+    """Times nosa_step on the workload `cfg` (args: steps, warmup, e2e_steps, launch); returns
+    the JSON line's fields on rank 0, None on the other ranks."""
     import torch
-    import torch.distributed as dist
     import kv_cache_offload_nosa_b200 as nosa
-    from kv_cache_offload_nosa_b200 import build as nb
     from kv_cache_offload_nosa_b200 import dist as D
 
-    rank, world, local = D.rank_info()
-    torch.cuda.set_device(local)
-    D.init("nccl", timeout_s=300)
-    nb.build()
     # each rank is an independent replica with its own seeded batch (weak scaling)
     if world > 1:
         cfg = cfg.with_(cfg_id=cfg.cfg_id + 1000 * rank)
@@ -309,7 +331,16 @@ def run_gpu(args, cfg):
     h_kn = torch.from_numpy(inp.k_new).view(torch.int16)
     h_vn = torch.from_numpy(inp.v_new).view(torch.int16)
     h_ev = torch.from_numpy(inp.evict)
-    d_q, d_kn, d_vn, d_ev = (x.cuda() for x in (h_q, h_kn, h_vn, h_ev))
+    def per_step(x):
+        # one row per step, each row starting on a 16-byte boundary (the library's alignment)
+        flat = x.reshape(x.shape[0], -1)
+        n = flat.shape[1]
+        per = 16 // flat.element_size()
+        d = torch.zeros((flat.shape[0], -(-n // per) * per), dtype=flat.dtype, device="cuda")
+        d[:, :n].copy_(flat)
+        return d[:, :n]
+
+    d_q, d_kn, d_vn, d_ev = (per_step(x) for x in (h_q, h_kn, h_vn, h_ev))
     sel = torch.empty(NG * cfg.k, dtype=torch.int32, device="cuda")
     out = torch.empty(cfg.B * cfg.Hq * cfg.d, dtype=torch.float32, device="cuda")
     # every step writes its miss counts to its own row (nothing extra runs in the timed region)
@@ -531,9 +562,7 @@ def run_gpu(args, cfg):
     # max over ranks
     tot_ms, e2e_ms = D.max_over_ranks([tot_ms, e2e_ms], device="cuda")
     if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
-        return
+        return None
     q_per_step = cfg.B * cfg.Hq * world
     value = q_per_step * args.steps / (tot_ms / 1e3)
     hbm_peak, peak_kind = peaks()
@@ -598,30 +627,20 @@ def run_gpu(args, cfg):
     if visited is not None:
         line["early_stop"] = {"tau": cfg.stop_tau, "blocks_streamed_per_group": visited, "k": cfg.k,
                               "kernel": "attn_stop_kernel (one CTA per group)"}
-    if not args.no_cpu_baseline:
-        cb, _ = oracle_sample(workload(args.workload, 4), 3, budget_s=args.cpu_budget)
-        line["cpu_baseline"] = cb
-    print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    return line
 
 
 # ----------------------------------------------------------------------------- lookahead
-def run_lookahead(args, cfg):
+def measure_lookahead(args, cfg, rank, world, local):
     """Tokens through `--layers` offload layers (independent caches of the workload's shape):
     SparDA's lookahead pipeline (plans ahead, layer-ordered copies on their own stream,
     attention after each layer's copies) against the same layers stepped one after another
     with nosa_step. Reports both token times and the time the pipeline hides."""
     import torch
     import kv_cache_offload_nosa_b200 as nosa
-    from kv_cache_offload_nosa_b200 import build as nb
     from kv_cache_offload_nosa_b200 import dist as D
     from kv_cache_offload_nosa_b200.lookahead import LookaheadPipeline
 
-    rank, world, local = D.rank_info()
-    torch.cuda.set_device(local)
-    D.init("nccl", timeout_s=300)
-    nb.build()
     nl = args.layers
     total = 2 * (args.warmup + args.steps) + 1
     cfgs = [cfg.with_(cfg_id=cfg.cfg_id + 1000 * l + 100000 * rank, steps=total) for l in range(nl)]
@@ -702,9 +721,7 @@ def run_lookahead(args, cfg):
     pcie_peak = pcie_ceiling(nosa, torch)
     tok_ms, ser_tok_ms = D.max_over_ranks([float(np.sum(pipe_ms)), float(np.sum(ser_ms))], device="cuda")
     if rank != 0:
-        if world > 1:
-            torch.distributed.destroy_process_group()
-        return
+        return None
     tok = tok_ms / args.steps
     ser = ser_tok_ms / args.steps
     page = cfg.block * cfg.d * 2
@@ -728,7 +745,75 @@ def run_lookahead(args, cfg):
         "gpu_launches": args.steps * nl * 4,
         "clocks": clk.summary(),
     }
-    print(json.dumps(line), flush=True)
+    return line
+
+
+# ----------------------------------------------------------------------------- driver
+# Workloads measured after the headline in the same process (one GPU only), each at a few
+# steps: every configuration of the decode step besides the headline layer.
+PER_CONFIG = ("tiny", "offload", "sink", "sweep_T65536_b64_p1", "sweep_T65536_b64_p5",
+              "sweep_T65536_b64_p10", "llama_stop", "llama_kc16", "lookahead")
+
+
+def summarize(name: str, line: dict) -> dict:
+    """The per-configuration entry: step time, queries/s and the HBM (or PCIe) fraction."""
+    if name == "lookahead":
+        keys = ("token_us", "serial_token_us", "hidden_us", "speedup_vs_serial", "pcie")
+        e = {"workload": line["config"]["workload"], "queries_per_s": line["value"]}
+        e.update({k: line[k] for k in keys})
+        return e
+    e = {"workload": line["config"]["workload"], "step_us": line["step_us"],
+         "step_us_median": line["step_us_median"], "queries_per_s": line["value"],
+         "hbm_gbs": line["hbm_gbs"], "hbm_frac": line["hbm_frac"], "bytes_per_step": line["bytes_per_step"],
+         "kernel_us": line["kernel_us"], "roofline_frac": line["roofline"]["frac"],
+         "roofline_kernel": line["roofline"]["kernel"], "step0_us": line["step0_us"],
+         "launch": line["launch"], "clocks": line["clocks"]}
+    for k in ("pcie", "early_stop"):
+        if k in line:
+            e[k] = line[k]
+    return e
+
+
+def per_config(args, rank, world, local):
+    import copy
+    import torch
+    out = {}
+    for name in PER_CONFIG:
+        a = copy.copy(args)
+        a.steps, a.warmup, a.e2e_steps = args.per_config_steps, 3, 4
+        a.no_cpu_baseline = True
+        cfg = workload(name, a.warmup + a.steps)
+        t0 = time.perf_counter()
+        try:
+            fn = measure_lookahead if name == "lookahead" else measure_gpu
+            line = fn(a, cfg, rank, world, local)
+            out[name] = summarize(name, line)
+        except Exception as e:  # one configuration's failure must not lose the headline line
+            out[name] = {"error": f"{type(e).__name__}: {str(e)[:300]}"}
+        out[name]["wall_s"] = time.perf_counter() - t0
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_gpu(args, cfg):
+    import torch
+    from kv_cache_offload_nosa_b200 import build as nb
+    from kv_cache_offload_nosa_b200 import dist as D
+
+    rank, world, local = D.rank_info()
+    torch.cuda.set_device(local)
+    D.init("nccl", timeout_s=300)
+    nb.build()
+    fn = measure_lookahead if cfg.name == "lookahead" else measure_gpu
+    line = fn(args, cfg, rank, world, local)
+    if rank == 0:
+        torch.cuda.empty_cache()
+        if cfg.name != "lookahead" and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args)
+        if world == 1 and args.per_config_steps > 0 and cfg.name == "llama" and not args.batch:
+            line["per_config"] = per_config(args, rank, world, local)
+        print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
 
@@ -747,14 +832,15 @@ def main():
     ap.add_argument("--layers", type=int, default=4, help="layers of the lookahead workload")
     ap.add_argument("--launch", default="graph", choices=["graph", "direct"],
                     help="timed steps as one replayed CUDA graph per step, or direct launches")
+    ap.add_argument("--per-config-steps", type=int, default=10,
+                    help="timed steps of each other workload measured after the headline "
+                         "(one GPU, default workload only); 0 = none")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = workload(args.workload, args.warmup + args.steps, args.batch)
     if args.impl == "reference":
         run_reference(args, cfg)
-    elif cfg.name == "lookahead" and args.impl == "native":
-        run_lookahead(args, cfg)
     else:
         run_gpu(args, cfg)
 

@@ -12,13 +12,14 @@
 //
 // Inside a CTA: one producer warp issues TMA tile loads (128-byte swizzle, no
 // multicast) of the K and V page of each task into a ring of shared-memory
-// stages; BS/16 consumer warps each own 16 tokens of every page. Per warp the
-// G query heads are rows 0..G-1 of an m16n8k16 bf16 mma (other rows zero);
-// q.K^T uses K straight from shared memory (ldmatrix). P.V uses V through
-// ldmatrix.trans with P split into bf16 hi + lo parts (a single bf16 P would
-// cost ~1e-3 relative error): rows 0..7 of the A operand carry P_hi and rows
-// 8..15 carry P_lo, so one mma accumulates both and the two halves of the
-// accumulator are summed when the partial is written.
+// stages; BS/16 consumer warps each own 16 tokens of every page. Those 16
+// tokens are the M side of both m16n8k16 bf16 products (K . q^T, then
+// V^T . P^T), the group's query heads the 8 N columns: a group supplies only
+// G <= 8 query rows, so with the tokens on M no row of a tile is padding. P is
+// split into bf16 high + low parts (a single bf16 P would cost ~1e-3 relative
+// error); with G <= 4 each head takes two columns, one per part, so a single
+// product accumulates both, and the parts are summed when the partial is
+// written.
 #pragma once
 
 #include "nosa_common.cuh"
@@ -82,8 +83,8 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
                 AttnArgs a) {
   using SH = AttnShape<D, BS>;
   constexpr int NC = SH::NC;
-  constexpr int NT = D / 8;     // 8-column n-tiles of the output
-  constexpr int KS = D / 16;    // 16-wide k-steps of q.K^T
+  constexpr int MT = D / 16;    // 16-dim m-tiles of the output (O^T)
+  constexpr int KS = D / 16;    // 16-wide k-steps of K.Qc
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int ST = a.stages;
@@ -198,11 +199,25 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
   }
 
   // ---------------------------------------------------------------- consumers
-  const int hrow = lane >> 2, c4 = lane & 3;
-  const bool row_ok = hrow < a.G;
-  uint32_t qa[KS][2];
-  float acc[NT][4];
-  float m_run = -INFINITY, l_run = 0.f;
+  // Per warp, the 16 tokens it owns in every page are the M rows of both products:
+  //   S^T  = K . Qc      A: K rows straight from shared memory (ldmatrix),
+  //                      B: Qc, the group's query heads as 8 columns;
+  //   O^T += V^T . P^T   A: V rows through ldmatrix.trans,
+  //                      B: P^T, put in place from the S^T accumulator layout by movmatrix.trans.
+  // With G <= 4 every head fills two columns, h and h + 4: column h carries the high bf16 part
+  // of P and column h + 4 the low part (P - high), so one product accumulates both and the
+  // halves are added when the partial is written. With G = 8 a second product adds the low parts.
+  const int r = lane >> 2, c4 = lane & 3;
+  const bool wide = a.G > 4;
+  auto col_head = [&](int n) { return wide ? n : (n & 3); };
+  const int h0 = col_head(2 * c4), h1 = col_head(2 * c4 + 1);  // heads of this lane's columns
+  const bool cv0 = h0 < a.G, cv1 = h1 < a.G;
+  const bool lo_cols = !wide && c4 >= 2;                       // columns 4..7: low parts
+  const bool owner = !wide ? c4 < 2 : true;                    // writes its columns' results
+  const int qhead = col_head(r);                               // B column r of Qc
+  uint32_t qb[KS][2];
+  float acc[MT][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;    // columns 2*c4 and 2*c4 + 1
   int cur = -1;
 
   for (int i = 0; i < ntask; ++i) {
@@ -217,16 +232,17 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
     if (ti.gi != cur) {
       cur = ti.gi;
       const int b = cur / a.Hkv, g = cur % a.Hkv;
-      const uint16_t* qrow = a.q + ((size_t)b * a.Hq + g * a.G + hrow) * D;
+      const bool qok = qhead < a.G;
+      const uint16_t* qrow = a.q + ((size_t)b * a.Hq + g * a.G + (qok ? qhead : 0)) * D;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        qa[ks][0] = row_ok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c4) : 0u;
-        qa[ks][1] = row_ok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c4) : 0u;
+        qb[ks][0] = qok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c4) : 0u;
+        qb[ks][1] = qok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c4) : 0u;
       }
 #pragma unroll
-      for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-      m_run = -INFINITY;
-      l_run = 0.f;
+      for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
     }
     bool wrote_smem = false, released = false;
     const int tok0 = ti.j * BS + 16 * warp;
@@ -241,76 +257,79 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
         wrote_smem = true;
         __syncwarp();
       }
-      // S = Q K^T for 16 tokens: two n-tiles of 8 tokens
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      {
-        const int mi = lane >> 3, r8 = lane & 7;
-        const int row = 16 * warp + 8 * (mi >> 1) + r8;
-        const uint32_t kbase = smem_u32(kst);
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kbase + swz<BS>(row, 16 * ks + 8 * (mi & 1)), b0, b1, b2, b3);
-          mma_16816(sc[0], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
-          mma_16816(sc[1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
-        }
-      }
-      // online softmax (log2 domain); row hrow, tokens 8*nt + 2*c4 + e
-      float p[2][2];
-      float mx = -INFINITY;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tk = 8 * nt + 2 * c4 + e;
-          const float v = (row_ok && tk < nval) ? sc[nt][e] * a.scale_log2 : -INFINITY;
-          p[nt][e] = v;
-          mx = fmaxf(mx, v);
-        }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m_run, mx);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = (m_new != m_run) ? ex2(m_run - m_use) : 1.f;
-      float psum = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          p[nt][e] = ex2(p[nt][e] - m_use);
-          psum += p[nt][e];
-        }
-      l_run = l_run * alpha + psum;
-      // the running max of most rows stops moving after the first blocks: rescale only when
-      // some row's max changed (alpha == 1 exactly otherwise)
-      const bool moved = m_new != m_run;
-      m_run = m_new;
-      if (__any_sync(0xffffffffu, moved)) {
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          acc[n][0] *= alpha;
-          acc[n][1] *= alpha;
-          acc[n][2] *= alpha;
-          acc[n][3] *= alpha;
-        }
-      }
-      // P as bf16 hi + lo (A operand rows = heads, k = 16 tokens)
-      const uint32_t ah0 = pack_bf16(p[0][0], p[0][1]);
-      const uint32_t ah2 = pack_bf16(p[1][0], p[1][1]);
-      const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&ah0);
-      const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&ah2);
-      const uint32_t al0 = pack_bf16(p[0][0] - __low2float(h0), p[0][1] - __high2float(h0));
-      const uint32_t al2 = pack_bf16(p[1][0] - __low2float(h2), p[1][1] - __high2float(h2));
+      // S^T for 16 tokens x 8 columns; two accumulators halve the dependent mma chain
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
       {
         const int mi = lane >> 3, r8 = lane & 7;
         const int row = 16 * warp + 8 * (mi & 1) + r8;
+        const uint32_t kbase = smem_u32(kst);
+#pragma unroll
+        for (int ks = 0; ks < KS; ks += 2) {
+          uint32_t x0, x1, x2, x3, y0, y1, y2, y3;
+          ldsm_x4(kbase + swz<BS>(row, 16 * ks + 8 * (mi >> 1)), x0, x1, x2, x3);
+          ldsm_x4(kbase + swz<BS>(row, 16 * ks + 16 + 8 * (mi >> 1)), y0, y1, y2, y3);
+          mma_16816(sa, x0, x1, x2, x3, qb[ks][0], qb[ks][1]);
+          mma_16816(sb, y0, y1, y2, y3, qb[ks + 1][0], qb[ks + 1][1]);
+        }
+      }
+      // online softmax (log2 domain) per column; this lane: tokens r and r + 8
+      const bool t0 = r < nval, t1 = r + 8 < nval;
+      const float x0 = (cv0 && t0) ? (sa[0] + sb[0]) * a.scale_log2 : -INFINITY;
+      const float x1 = (cv1 && t0) ? (sa[1] + sb[1]) * a.scale_log2 : -INFINITY;
+      const float x2 = (cv0 && t1) ? (sa[2] + sb[2]) * a.scale_log2 : -INFINITY;
+      const float x3 = (cv1 && t1) ? (sa[3] + sb[3]) * a.scale_log2 : -INFINITY;
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0, mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+      const float al0 = (mn0 != m0) ? ex2(m0 - mu0) : 1.f;
+      const float al1 = (mn1 != m1) ? ex2(m1 - mu1) : 1.f;
+      const float p0 = ex2(x0 - mu0), p2 = ex2(x2 - mu0);
+      const float p1 = ex2(x1 - mu1), p3 = ex2(x3 - mu1);
+      l0 = l0 * al0 + (p0 + p2);
+      l1 = l1 * al1 + (p1 + p3);
+      // the running max of most columns stops moving after the first blocks: rescale only
+      // when some column's max changed (alpha == 1 exactly otherwise)
+      const bool moved = (mn0 != m0) || (mn1 != m1);
+      m0 = mn0;
+      m1 = mn1;
+      if (__any_sync(0xffffffffu, moved)) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          acc[mt][0] *= al0;
+          acc[mt][1] *= al1;
+          acc[mt][2] *= al0;
+          acc[mt][3] *= al1;
+        }
+      }
+      // P as bf16 high + low parts, in the S^T layout (rows = tokens r / r + 8)
+      const uint32_t hi01 = pack_bf16(p0, p1), hi23 = pack_bf16(p2, p3);
+      const __nv_bfloat162 e01 = *reinterpret_cast<const __nv_bfloat162*>(&hi01);
+      const __nv_bfloat162 e23 = *reinterpret_cast<const __nv_bfloat162*>(&hi23);
+      const uint32_t lo01 = pack_bf16(p0 - __low2float(e01), p1 - __high2float(e01));
+      const uint32_t lo23 = pack_bf16(p2 - __low2float(e23), p3 - __high2float(e23));
+      // P^T as the B operand: column n = lane >> 2, tokens 2*c4.. (b0) and 8 + 2*c4.. (b1)
+      const uint32_t pb0 = movmatrix_t(lo_cols ? lo01 : hi01);
+      const uint32_t pb1 = movmatrix_t(lo_cols ? lo23 : hi23);
+      uint32_t pl0 = 0u, pl1 = 0u;
+      if (wide) {
+        pl0 = movmatrix_t(lo01);
+        pl1 = movmatrix_t(lo23);
+      }
+      {
+        const int mi = lane >> 3, r8 = lane & 7;
+        const int row = 16 * warp + 8 * (mi >> 1) + r8;
         const uint32_t vbase = smem_u32(vst);
 #pragma unroll
-        for (int np = 0; np < NT / 2; ++np) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(vbase + swz<BS>(row, 16 * np + 8 * (mi >> 1)), b0, b1, b2, b3);
-          mma_16816(acc[2 * np], ah0, al0, ah2, al2, b0, b1);
-          mma_16816(acc[2 * np + 1], ah0, al0, ah2, al2, b2, b3);
+        for (int mt = 0; mt < MT; ++mt) {
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_t(vbase + swz<BS>(row, 16 * mt + 8 * (mi & 1)), v0, v1, v2, v3);
+          mma_16816(acc[mt], v0, v1, v2, v3, pb0, pb1);
+          if (wide) mma_16816(acc[mt], v0, v1, v2, v3, pl0, pl1);
         }
       }
     }
@@ -318,20 +337,43 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
     if (ti.last) {
       // ------------------------------------------------ flush this group's part
       named_bar(1, NC * 32);  // every consumer is done reading stage s
-      float l = l_run;
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      float L0 = l0, L1 = l1;  // sums over the warp's 16 token rows
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        L0 += __shfl_xor_sync(0xffffffffu, L0, o);
+        L1 += __shfl_xor_sync(0xffffffffu, L1, o);
+      }
+      if (!wide) {
+        // high part (columns 0..3, lanes c4 < 2) + low part (columns 4..7, lanes c4 + 2)
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[mt][e] += __shfl_xor_sync(0xffffffffu, acc[mt][e], 2);
+      }
       float* scr = reinterpret_cast<float*>(kst);  // [NC][G][D+2] in the spent stage
-      if (row_ok) {
-        float* w = scr + ((size_t)warp * a.G + hrow) * (D + 2);
-        if (c4 == 0) {
-          w[0] = m_run;
-          w[1] = l;
+      if (owner) {
+        float* w0 = scr + ((size_t)warp * a.G + h0) * (D + 2);
+        float* w1 = scr + ((size_t)warp * a.G + h1) * (D + 2);
+        if (r == 0) {
+          if (cv0) {
+            w0[0] = m0;
+            w0[1] = L0;
+          }
+          if (cv1) {
+            w1[0] = m1;
+            w1[1] = L1;
+          }
         }
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          w[2 + 8 * n + 2 * c4] = acc[n][0] + acc[n][2];
-          w[3 + 8 * n + 2 * c4] = acc[n][1] + acc[n][3];
+        for (int mt = 0; mt < MT; ++mt) {
+          if (cv0) {
+            w0[2 + 16 * mt + r] = acc[mt][0];
+            w0[2 + 16 * mt + 8 + r] = acc[mt][2];
+          }
+          if (cv1) {
+            w1[2 + 16 * mt + r] = acc[mt][1];
+            w1[2 + 16 * mt + 8 + r] = acc[mt][3];
+          }
         }
       }
       wrote_smem = true;

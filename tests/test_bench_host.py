@@ -93,23 +93,34 @@ def test_clock_summary_without_sampler():
 def test_traffic_record_needs_the_captured_source(tmp_path, monkeypatch):
     """The ncu traffic figure is reported only while the attention kernel's source hashes to
     the one that was captured, scaled from the captured batch by the number of groups."""
-    import hashlib
+    import json
     root = tmp_path / "r"
     csrc = root / "kv_cache_offload_nosa_b200" / "csrc"
     csrc.mkdir(parents=True)
     (root / "profiles").mkdir()
     for f in ("nosa_attn.cuh", "nosa_common.cuh"):
         shutil.copy(os.path.join(bench.ROOT, "kv_cache_offload_nosa_b200", "csrc", f), csrc / f)
-    h = hashlib.sha256()
-    for f in ("nosa_attn.cuh", "nosa_common.cuh"):
-        h.update((csrc / f).read_bytes())
-    (root / "profiles" / "attn_kernel_llama_b8.md").write_text(
-        f"traffic-record: batch=8 dram_bytes_per_launch=1000 source_sha256={h.hexdigest()}\n")
     monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.attn_traffic(16) is None  # no record
+    (root / "profiles" / "attn_traffic.json").write_text(json.dumps(
+        {"batch": 8, "dram_bytes_per_launch": 1000, "source_sha256": bench.kernel_source_sha()}))
     assert bench.attn_traffic(16) == 2000
     with open(csrc / "nosa_attn.cuh", "a") as f:
         f.write("// changed\n")
     assert bench.attn_traffic(16) is None
+
+
+def test_committed_traffic_record_is_well_formed():
+    """profiles/attn_traffic.json, when present, names its batch, bytes, source hash and the
+    ncu command it came from (which leaves the clocks alone)."""
+    import json
+    p = os.path.join(bench.ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(p):
+        pytest.skip("no traffic record committed")
+    rec = json.load(open(p))
+    assert rec["batch"] > 0 and rec["dram_bytes_per_launch"] > 0
+    assert len(rec["source_sha256"]) == 64
+    assert "--clock-control none" in rec["command"]
 
 
 def test_profile_commands_leave_clocks_alone_and_run_committed_files():

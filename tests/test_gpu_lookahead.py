@@ -60,14 +60,16 @@ def test_lookahead_on_side_streams():
         H.compare_step(cache, cfg, rec, io, t)
 
 
-def test_lookahead_pipeline_two_layers():
-    """LookaheadPipeline over two layers (independent caches): each layer equals its own
-    oracle run."""
+@pytest.mark.parametrize("layers", [2, 4])
+def test_lookahead_pipeline_layers(layers):
+    """LookaheadPipeline over several layers (independent caches): each layer equals its own
+    oracle run. With 4 layers the plans of layers 2 and 3 wait for the attention of layers 0
+    and 1 (their forecast rows' inputs) on another stream."""
     _need_gpu()
     import gpu_harness as H
     from kv_cache_offload_nosa_b200.lookahead import LookaheadPipeline
     base = CS["lookahead_small"]
-    cases = [O.run_case(base.with_(cfg_id=base.cfg_id + 1000 * l), lookahead=True) for l in range(2)]
+    cases = [O.run_case(base.with_(cfg_id=base.cfg_id + 1000 * l), lookahead=True) for l in range(layers)]
     caches = [H.setup(c.cfg, c.inputs) for c in cases]
     ios = [H.StepIO(c.cfg) for c in cases]
     pipe = LookaheadPipeline(caches)
