@@ -117,7 +117,7 @@ nosa_status check_state(const nosa_config& c, const nosa_state* st) {
 
 struct WsLayout {
   size_t scores, cnt_k1, cnt_attn, copy_list, copy_count, partials, ge_mask, sel_flag, copy_cnt,
-      copy_flag, units, used, total;
+      copy_flag, units, used, att_list, e_flag, total;
   int copy_stride;
 };
 
@@ -143,6 +143,8 @@ WsLayout ws_layout(const nosa_config& c) {
   const size_t urows = !c.score_mode ? 0 : ((c.score_mode & NOSA_SCORE_SOFTMAX) ? c.n_score_rows : 1);
   w.units = off; off += up256(NG * urows * (size_t)max_sub(c) * 4);
   w.used = off; off += up256((size_t)c.B * c.Hq * 4);
+  w.att_list = off; off += up256(NG * (size_t)kk(c) * 4);
+  w.e_flag = off; off += up256(NG * kFlagStride * 4);
   w.total = off;
   return w;
 }
@@ -202,12 +204,34 @@ void set_ws(StepArgs& a, const nosa_config& c, void* ws) {
 }
 
 // ------------------------------------------------------------------ launches
+// Score CTAs of 256 sub-blocks: about three waves on the Llama-shaped layer, each CTA short
+// enough that an SM's CTAs finish at staggered times. (Larger chunks, one wave of about two CTAs
+// per SM, streamed slower: fewer loads in flight.)
+constexpr int kScoreChunk = 256;
+// Shared-memory carveout (percent) of the score kernel, or -1 for the driver's choice, and the
+// attention's shared memory for tile stages (its carveout is the largest shared split).
+constexpr int kStepCarveout = -1;
+constexpr int kAttnStageBudget = 110 * 1024;
+// The fused step publishes each group's query-agnostic blocks ahead of the rest of its selection.
+constexpr bool kEarlyGammaE = true;
+
+nosa_status score_chunk(const nosa_config& c, int* chunk) {
+  (void)c;
+  *chunk = kScoreChunk;
+  return NOSA_OK;
+}
+
 template <int D, bool FUSED, int VARIANT, bool KC16>
-nosa_status launch_score_t(const nosa_config& c, const StepArgs& a, cudaStream_t s) {
-  dim3 grid((max_sub(c) + kChunkSub - 1) / kChunkSub, n_groups(c));
-  const size_t dsm = FUSED ? sel_smem_bytes(c.max_blocks) : 0;
+nosa_status launch_score_t(const nosa_config& c, const StepArgs& a0, cudaStream_t s) {
+  StepArgs a = a0;
+  nosa_status r = score_chunk(c, &a.chunk);
+  if (r != NOSA_OK) return r;
+  dim3 grid((max_sub(c) + a.chunk - 1) / a.chunk, n_groups(c));
+  const size_t dsm = (FUSED ? score_su_offset(c.max_blocks) : 0) + (size_t)a.chunk * 4;
   auto k = score_kernel<D, FUSED, VARIANT, KC16>;
   if (dsm > 48 * 1024) NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm));
+  if (kStepCarveout >= 0)
+    NOSA_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, kStepCarveout));
   k<<<grid, kScoreThreads, dsm, s>>>(a);
   NOSA_CUDA(cudaGetLastError());
   return NOSA_OK;
@@ -320,7 +344,7 @@ template <int D, int BS>
 nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& tk, const CUtensorMap& tv,
                           cudaStream_t s, bool finest, bool pdl = true) {
   using SH = AttnShape<D, BS>;
-  int stages = (110 * 1024) / SH::STAGE;
+  int stages = kAttnStageBudget / SH::STAGE;
   stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
   const size_t smem = SH::smem_bytes(stages);
   auto k = attn_kernel<D, BS>;
@@ -445,15 +469,21 @@ nosa_status dispatch_attn(const nosa_config& c, const AttnArgs& a, const CUtenso
 
 // ready: per-group flags the attention waits on (and clears), or NULL to wait for the
 // previous grid as a whole. pdl: may start while the previous kernel on the stream runs.
+// early: the score kernel of the same step publishes each group's query-agnostic blocks
+// ahead of the rest of its selection (per-group flags only).
 nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16_t* q, const int32_t* sel,
                         float* out, void* ws, cudaStream_t s, uint32_t* ready = nullptr,
-                        bool pdl = true) {
+                        bool pdl = true, bool early = false) {
   CUtensorMap tk, tv;
   nosa_status r = make_pool_maps(c, st, &tk, &tv);
   if (r != NOSA_OK) return r;
   const WsLayout w = ws_layout(c);
   AttnArgs a = attn_args(c, st, q, sel, out, ws_at<float>(ws, w.partials), ws_at<uint32_t>(ws, w.cnt_attn));
   a.sel_flag = ready;
+  if (early && ready) {
+    a.att_list = ws_at<int32_t>(ws, w.att_list);
+    a.e_flag = ws_at<uint32_t>(ws, w.e_flag);
+  }
   if (c.stop_tau > 0.f) {
     // early stop: one CTA per group, after the whole previous grid (no per-group flags)
     StopArgs x;
@@ -693,13 +723,18 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   // early stop waits for the previous grid as a whole: no per-group flags then
   const bool flags = !events && !(c.stop_tau > 0.f);
   a.sel_flag = flags ? ws_at<uint32_t>(ws, w.sel_flag) : nullptr;
+  if (flags && kEarlyGammaE) {
+    // the query-agnostic blocks of a group are attended as soon as they are chosen
+    a.att_list = ws_at<int32_t>(ws, w.att_list);
+    a.e_flag = ws_at<uint32_t>(ws, w.e_flag);
+  }
   uint32_t* ready = !flags ? nullptr
                            : ws_at<uint32_t>(ws, has_host(st) ? w.copy_flag : w.sel_flag);
   if ((r = launch_score<true>(c, a, s)) != NOSA_OK) return r;
   if ((r = rec(1)) != NOSA_OK) return r;
   if (has_host(st) && (r = launch_copy(c, st, ws, s, flags)) != NOSA_OK) return r;
   if ((r = rec(2)) != NOSA_OK) return r;
-  if ((r = launch_attn(c, st, q, sel, out, ws, s, ready)) != NOSA_OK) return r;
+  if ((r = launch_attn(c, st, q, sel, out, ws, s, ready, true, flags && kEarlyGammaE)) != NOSA_OK) return r;
   return rec(3);
 }
 

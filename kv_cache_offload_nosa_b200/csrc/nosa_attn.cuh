@@ -44,13 +44,18 @@ struct AttnArgs {
   long long total_pages;
   float scale_log2;           // sigma * log2(e)
   uint32_t* sel_flag;         // [B*Hkv * kFlagStride] per-group "ready" flags, or NULL
+  // early start (with sel_flag): the task order and the early flags the score kernel
+  // publishes (Gamma_e first, then Gamma_q; see StepArgs), or NULL to read sel and seq_len
+  const int32_t* att_list;    // [B*Hkv][k]
+  uint32_t* e_flag;           // [B*Hkv * kFlagStride]: [0] flag, [1] L, [2] |Gamma_e|
   int identity;               // no host pools: block j of group g is page g * max_blocks + j
                               // (the state's block table is that identity), so no lookup
   unsigned long long wait_ns; // limit of every bounded wait, from the kernel's start
 };
 
 struct TaskInfo {
-  int gi, j, L, last;
+  int gi, j, L, last;         // gi < 0: no more tasks
+  int seg, nseg;              // the task's partial slot in its group, and the group's slot count
 };
 
 template <int D, int BS>
@@ -78,7 +83,9 @@ __device__ __forceinline__ uint32_t swz(int row, int col) {
 }
 
 template <int D, int BS>
-__global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
+// (3 CTAs per SM for register allocation: 136 registers or fewer at 64-token blocks, so one
+// attention CTA fits beside two score CTAs while the step's score kernel still runs)
+__global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 3)
     attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 AttnArgs a) {
   using SH = AttnShape<D, BS>;
@@ -116,81 +123,126 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
 
   if (warp == NC) {
     // ---------------------------------------------------------------- producer
-    // The warp resolves 32 tasks' metadata at once (sel -> block table, in parallel
-    // across lanes); lane 0 then issues the tile loads in task order.
-    int issued = 0;
+    // The CTA's W tasks are cut at group boundaries into ranges, each ending in a partial
+    // (m, l, acc) slot of its group. A range is taken in parts that wait for the same flag:
+    // with early publication a group's first |Gamma_e| positions (its query-agnostic blocks,
+    // with the context length) are ready before the query-aware selection, the rest once the
+    // whole selection (and, with host pools, its page copies) is in place. Per part the warp
+    // resolves 32 tasks' metadata at once (block -> page, in parallel across lanes); lane 0
+    // then issues the tile loads in task order. Lane 0 acquires each flag; the warp barrier
+    // orders the other lanes' loads (L2, __ldcg) after that acquire.
+    const bool early = a.att_list != nullptr;
+    const int32_t* list = early ? a.att_list : a.sel;
+    int it = 0;  // tasks issued (stage ring position)
     bool abort = false;
-    for (int base = 0; base < ntask && !abort; base += 32) {
-      const int i_l = base + lane;
-      int gi_l = 0, j_l = -1, L_l = 0, page_l = -1;
-      if (flags) {
-        // lane 0 acquires the flags of the batch's groups (contiguous, in order); the warp
-        // barrier orders the other lanes' loads below (L2, __ldcg) after those acquires
-        if (lane == 0) {
-          const int g1 = (task0 + min(base + 32, ntask) - 1) / a.k;
-          for (int g = (task0 + base) / a.k; g <= g1; ++g)
-            if (!wait_flag(a.sel_flag + (size_t)g * kFlagStride, deadline)) set_err(a.err, NOSA_ERR_TIMEOUT);
-        }
-        __syncwarp();
-      }
-      if (i_l < ntask) {
-        const int t = task0 + i_l;
-        gi_l = t / a.k;
-        L_l = __ldcg(a.seq_len + gi_l);
-        const int N = (L_l + BS - 1) / BS;
-        j_l = __ldcg(a.sel + t);
-        if (j_l >= N) {
-          set_err(a.err, NOSA_ERR_SEL);
-          j_l = -1;
-        }
-        if (j_l >= 0) {
-          page_l = a.identity ? gi_l * a.max_blocks + j_l
-                              : __ldcg(a.block_table + (size_t)gi_l * a.max_blocks + j_l);
-          if (page_l < 0 || page_l >= a.total_pages) {
-            set_err(a.err, NOSA_ERR_BLOCK_TABLE);
-            j_l = -1;
+    for (int sr = 0; sr < ntask && !abort;) {
+      // the group, the positions [pa, pb) of its order in this CTA, and the partial slot
+      const int gi = (task0 + sr) / a.k;
+      const int pa = task0 + sr - gi * a.k;
+      const int pb = min(task0 + ntask, (gi + 1) * a.k) - gi * a.k;
+      const int first = (int)(((long long)gi * a.k) / a.W);
+      const int lastc = (int)(((long long)gi * a.k + a.k - 1) / a.W);
+      const int seg = blockIdx.x - first, nseg = lastc - first + 1;
+      sr += pb - pa;
+      const int tbase = gi * a.k;  // task index of the group's position 0
+      for (int p = pa; p < pb && !abort;) {
+        int pend = pb, L;
+        const uint32_t* f = flags ? a.sel_flag + (size_t)gi * kFlagStride : nullptr;
+        if (early) {
+          const uint32_t* ef = a.e_flag + (size_t)gi * kFlagStride;
+          if (lane == 0 && !wait_flag(ef, deadline)) set_err(a.err, NOSA_ERR_TIMEOUT);
+          __syncwarp();
+          L = static_cast<int>(__ldcg(ef + 1));
+          const int ne = static_cast<int>(__ldcg(ef + 2));
+          if (p < ne) {  // query-agnostic part: ready now
+            pend = min(pb, ne);
+            f = nullptr;
           }
         }
-      }
-      const int nb = min(32, ntask - base);
-      __syncwarp();
-      if (flags && lane == 0) fence_proxy_async_global();  // pages written before the flags
-      for (int u = 0; u < nb; ++u) {
-        const int gi = __shfl_sync(0xffffffffu, gi_l, u);
-        const int j = __shfl_sync(0xffffffffu, j_l, u);
-        const int L = __shfl_sync(0xffffffffu, L_l, u);
-        const int page = __shfl_sync(0xffffffffu, page_l, u);
-        const int i = base + u;
-        if (lane == 0) {
-          const int s = i % ST, round = i / ST;
-          if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, deadline)) {
-            set_err(a.err, NOSA_ERR_TIMEOUT);
-            abort = true;
-          } else {
-            TaskInfo ti;
-            ti.gi = gi;
-            ti.j = j;
-            ti.L = L;
-            ti.last = (i == ntask - 1) || ((task0 + i + 1) / a.k != gi);
-            info[s] = ti;
-            if (j >= 0) {
-              mbar_arrive_expect_tx(&full[s], SH::STAGE);
-              uint8_t* st = smem + (size_t)s * SH::STAGE;
-#pragma unroll
-              for (int h = 0; h < SH::HALVES; ++h) {
-                tma_load_2d(st + h * SH::TILE, &tmk, &full[s], 64 * h, page * BS);
-                tma_load_2d(st + SH::KV + h * SH::TILE, &tmv, &full[s], 64 * h, page * BS);
-              }
-            } else {
-              mbar_arrive(&full[s]);
+        if (f) {
+          if (lane == 0 && !wait_flag(f, deadline)) set_err(a.err, NOSA_ERR_TIMEOUT);
+          __syncwarp();
+        }
+        if (!early) L = __ldcg(a.seq_len + gi);
+        if (flags && lane == 0) fence_proxy_async_global();  // pages written before the flags
+        const int N = (L + BS - 1) / BS;
+        for (int base = p; base < pend && !abort; base += 32) {
+          const int p_l = base + lane;
+          int j_l = -1, page_l = -1;
+          if (p_l < pend) {
+            j_l = __ldcg(list + tbase + p_l);
+            if (j_l >= N) {
+              set_err(a.err, NOSA_ERR_SEL);
+              j_l = -1;
             }
-            issued = i + 1;
+            if (j_l >= 0) {
+              page_l = a.identity ? gi * a.max_blocks + j_l
+                                  : __ldcg(a.block_table + (size_t)gi * a.max_blocks + j_l);
+              if (page_l < 0 || page_l >= a.total_pages) {
+                set_err(a.err, NOSA_ERR_BLOCK_TABLE);
+                j_l = -1;
+              }
+            }
+          }
+          const int nb = min(32, pend - base);
+          __syncwarp();
+          for (int v = 0; v < nb; ++v) {
+            const int j = __shfl_sync(0xffffffffu, j_l, v);
+            const int page = __shfl_sync(0xffffffffu, page_l, v);
+            if (lane == 0) {
+              const int s = it % ST, round = it / ST;
+              if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, deadline)) {
+                set_err(a.err, NOSA_ERR_TIMEOUT);
+                abort = true;
+              } else {
+                TaskInfo ti;
+                ti.gi = gi;
+                ti.j = j;
+                ti.L = L;
+                ti.last = (base + v == pb - 1);
+                ti.seg = seg;
+                ti.nseg = nseg;
+                info[s] = ti;
+                if (j >= 0) {
+                  mbar_arrive_expect_tx(&full[s], SH::STAGE);
+                  uint8_t* st = smem + (size_t)s * SH::STAGE;
+#pragma unroll
+                  for (int h = 0; h < SH::HALVES; ++h) {
+                    tma_load_2d(st + h * SH::TILE, &tmk, &full[s], 64 * h, page * BS);
+                    tma_load_2d(st + SH::KV + h * SH::TILE, &tmv, &full[s], 64 * h, page * BS);
+                  }
+                } else {
+                  mbar_arrive(&full[s]);
+                }
+                ++it;
+              }
+            }
+            abort = __shfl_sync(0xffffffffu, abort, 0);
+            if (abort) break;
           }
         }
-        abort = __shfl_sync(0xffffffffu, abort, 0);
-        if (abort) break;
+        p = pend;
       }
     }
+    // end of the CTA's tasks: a task with gi < 0 stops the consumers
+    if (lane == 0 && !abort) {
+      const int s = it % ST, round = it / ST;
+      if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, deadline)) {
+        set_err(a.err, NOSA_ERR_TIMEOUT);
+      } else {
+        TaskInfo ti;
+        ti.gi = -1;
+        ti.j = -1;
+        ti.L = 0;
+        ti.last = 0;
+        ti.seg = 0;
+        ti.nseg = 0;
+        info[s] = ti;
+        mbar_arrive(&full[s]);
+        ++it;
+      }
+    }
+    const int issued = it;
     // never leave the CTA with a tile load in flight
     if (lane == 0)
       for (int i = max(0, issued - ST); i < issued; ++i)
@@ -220,13 +272,14 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;    // columns 2*c4 and 2*c4 + 1
   int cur = -1;
 
-  for (int i = 0; i < ntask; ++i) {
+  for (int i = 0;; ++i) {
     const int s = i % ST;
     if (!mbar_wait(&full[s], (i / ST) & 1, deadline)) {
       set_err(a.err, NOSA_ERR_TIMEOUT);
       break;
     }
     const TaskInfo ti = info[s];
+    if (ti.gi < 0) break;  // the producer has no more tasks (nothing in this stage to release)
     uint8_t* kst = smem + (size_t)s * SH::STAGE;
     uint8_t* vst = kst + SH::KV;
     if (ti.gi != cur) {
@@ -379,10 +432,7 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
       wrote_smem = true;
       named_bar(1, NC * 32);
       const int gi = ti.gi;
-      const int first = (int)(((long long)gi * a.k) / a.W);
-      const int lastc = (int)(((long long)gi * a.k + a.k - 1) / a.W);
-      const int nseg = lastc - first + 1;
-      const int seg = blockIdx.x - first;
+      const int nseg = ti.nseg, seg = ti.seg;
       const int GE = a.G * (D + 2);
       float* part = a.partials + ((size_t)gi * kPartialSlots + seg) * GE;
       for (int e = tid; e < GE; e += NC * 32) {
@@ -434,9 +484,15 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, BS == 128 ? 1 : 2)
         if (tid == 0) {
           a.counters[gi] = 0u;
           if (flags) a.sel_flag[(size_t)gi * kFlagStride] = 0u;  // every CTA of the group passed its wait
+          if (a.e_flag) {
+            a.e_flag[(size_t)gi * kFlagStride] = 0u;
+            a.e_flag[(size_t)gi * kFlagStride + 3] = 0u;
+          }
         }
       }
       named_bar(1, NC * 32);
+      // the partial is written: the next task starts a new one
+      cur = -1;
     }
     if (!released) {
       if (wrote_smem) fence_proxy_async_smem();

@@ -23,7 +23,7 @@
 namespace nosa {
 
 constexpr int kScoreThreads = 256;
-constexpr int kChunkSub = 256;  // sub-blocks per score CTA
+constexpr int kChunkAlign = 64;  // a score CTA's sub-block count is a multiple of this
 
 struct StepArgs {
   // scoring
@@ -66,7 +66,13 @@ struct StepArgs {
   int kc16;               // kc holds bf16 means (else fp32)
   int mode;               // scoring variant bits (1 windows, 2 per-row softmax); 0 = NOSA pool
   float* units;           // variants: per-sub-block values [B*Hkv][rows][max_sub] (workspace)
+  int chunk;              // sub-blocks per score CTA (a multiple of kChunkAlign)
   unsigned long long wait_ns;  // limit of the bounded waits (append_kernel's flag)
+  // early publication of the query-agnostic set (fused step with per-group flags), or NULL:
+  int32_t* att_list;      // [B*Hkv][k] attention order: Gamma_e ascending, Gamma_q ascending, -1
+  uint32_t* e_flag;       // [B*Hkv * kFlagStride]: [0] set once Gamma_e is in att_list and the
+                          // step's token is in place, [1] the context length L after the
+                          // append, [2] the early part's length, [3] parties done (0..2)
 };
 
 constexpr int kMaxSoftRows = 8;  // scoring rows the per-row softmax variant supports
@@ -205,14 +211,15 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   constexpr int SPW = 32 / LPS;      // sub-blocks per warp pass
   constexpr int PASS = SPW * (kScoreThreads / 32);
   __shared__ float qbar[D];
-  __shared__ float su[kChunkSub];
   __shared__ int s_last;
   __shared__ float vred[VARIANT ? 2 * kMaxSoftRows + kMaxSoftRows * (kScoreThreads / 32) : 1];
   extern __shared__ __align__(16) uint8_t dsm[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gi = blockIdx.y, c = blockIdx.x;
-  const int i0 = c * kChunkSub;
+  const int i0 = c * a.chunk;
+  // dynamic shared memory: [selection scratch (fused)] [this chunk's sub-block values]
+  float* su = reinterpret_cast<float*>(dsm + (FUSED ? score_su_offset(a.max_blocks) : 0));
   const int sub = lane / LPS, part = lane % LPS;
   using Vec = typename std::conditional<KC16, uint4, float4>::type;
   constexpr int NV = KC16 ? 2 : 4;          // 16-byte loads per lane and sub-block row
@@ -223,7 +230,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
 
   if (FUSED) griddep_launch_dependents();  // the next kernel may start its prologue
   // first batch of kc loads goes out before anything that depends on seq_len
-  const int icap = min(i0 + kChunkSub, a.max_sub);
+  const int icap = min(i0 + a.chunk, a.max_sub);
   int base = i0 + warp * SPW;
   Vec va[NV], vb[NV];
   auto load_batch = [&](int bse, int lim, Vec* xa, Vec* xb) {
@@ -248,19 +255,47 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   const int M = (L + a.s - 1) / a.s;
   const int N = (L + a.bs - 1) / a.bs;
   const int spb = a.bs / a.s;
-  const int i1 = min(i0 + kChunkSub, M);
+  const int i1 = min(i0 + a.chunk, M);
   const int Wmax = (a.max_blocks + 31) / 32;
 
-  if (FUSED && c == 0) {
-    // query-agnostic selection needs no block score: it overlaps the other chunks' streaming
-    const SelSmem S = sel_smem_carve(dsm, a.max_blocks);
-    select_evict(S, a.evict + (size_t)gi * a.max_blocks, a.prev_sel + (size_t)gi * Wmax,
-                 a.alive + (size_t)gi * Wmax, a.ge_mask + (size_t)gi * Wmax, N, a.k_e, Wmax);
-  }
-  if (FUSED && L > len0 && (len0 / a.s) / kChunkSub == c) {
+  // The query-agnostic selection needs no block score: chunk 0 runs it while the other chunks
+  // stream. With early publication its blocks can be attended before the query-aware half is
+  // known (NOSA, "Seleccion Independiente de la Consulta": Gamma_e depends on the eviction
+  // scores only), once the step's token is in place too: chunk 0 and the chunk that appends
+  // each count themselves done, and the second publishes. Only Gamma_e's blocks already in
+  // HBM go early: Gamma_e lies in S(t-1), which the previous step made resident, but the
+  // first step after set-up starts from S(-1) = every prefill block and only the initial
+  // residency.
+  const int c_app = (FUSED && L > len0) ? (len0 / a.s) / a.chunk : -1;
+  const bool parties2 = c_app > 0;  // chunk 0 and another chunk share the publication
+  if (FUSED && c == c_app) {
     append_token<D>(a, gi, len0);
     __syncthreads();
     load_batch(base, icap, va, vb);  // the tail sub-block's mean just changed
+  }
+  if (FUSED && c == 0) {
+    const SelSmem S = sel_smem_carve(dsm, a.max_blocks);
+    select_evict(S, a.evict + (size_t)gi * a.max_blocks, a.prev_sel + (size_t)gi * Wmax,
+                 a.alive + (size_t)gi * Wmax, a.ge_mask + (size_t)gi * Wmax, N, a.k_e, Wmax);
+    if (a.e_flag) {
+      const int W = (N + 31) / 32;
+      resident_bits(S.ge, S.m2, a.host_k ? a.block_table + (size_t)gi * a.max_blocks : nullptr, W);
+      const int ne = sel_compact(S, S.m2, W, a.att_list + (size_t)gi * (a.k_q + a.k_e));
+      if (tid == 0) a.e_flag[(size_t)gi * kFlagStride + 2] = static_cast<uint32_t>(ne);
+    }
+  }
+  if (FUSED && a.e_flag && (c == 0 || c == c_app)) {
+    __syncthreads();  // this CTA's part (Gamma_e's list, or the appended token) is written
+    if (tid == 0) {
+      uint32_t* ef = a.e_flag + (size_t)gi * kFlagStride;
+      __threadfence();
+      const bool second = !parties2 || atomicAdd(ef + 3, 1u) == 1u;
+      if (second) {
+        __threadfence();
+        ef[1] = static_cast<uint32_t>(L);
+        st_release_gpu(ef, 1u);
+      }
+    }
   }
   for (int x = tid; x < D; x += kScoreThreads) {
     const uint16_t* r = a.rows + (size_t)gi * a.R * D + x;
@@ -382,8 +417,9 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   }
   // block max over present sub-blocks; -inf for blocks not yet created
   if (!VARIANT) {
-    const int j = i0 / spb + tid;
-    if (tid < kChunkSub / spb && j < a.max_blocks) {
+    for (int jj = tid; jj < a.chunk / spb; jj += kScoreThreads) {
+      const int j = i0 / spb + jj;
+      if (j >= a.max_blocks) break;
       float m = -INFINITY;
       if (j < N) {
         const int e = min((j + 1) * spb, M);
@@ -406,6 +442,19 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(StepArgs a) {
   const int k = a.k_q + a.k_e;
   select_query(S, a.block_scores + (size_t)gi * a.max_blocks, a.ge_mask + (size_t)gi * Wmax,
                a.prev_sel + (size_t)gi * Wmax, a.sel + (size_t)gi * k, N, k, Wmax);
+  if (a.e_flag) {
+    // the rest of the attention order after the early part (Gamma_e's resident blocks, found
+    // again from the same block table: nothing changes it before the residency plan below):
+    // S(t) minus that part ascending, then -1
+    const int W = (N + 31) / 32;
+    const int ne = static_cast<int>(__ldcg(a.e_flag + (size_t)gi * kFlagStride + 2));
+    resident_bits(S.ge, S.m2, a.host_k ? a.block_table + (size_t)gi * a.max_blocks : nullptr, W);
+    for (int w = tid; w < W; w += kScoreThreads) S.m1[w] = S.sset[w] & ~S.m2[w];
+    __syncthreads();
+    int32_t* al = a.att_list + (size_t)gi * k;
+    const int nr = sel_compact(S, S.m1, W, al + ne);
+    for (int i = ne + nr + tid; i < k; i += kScoreThreads) al[i] = -1;
+  }
   if (a.host_k) {
     PlanArgs p;
     p.block_table = a.block_table + (size_t)gi * a.max_blocks;

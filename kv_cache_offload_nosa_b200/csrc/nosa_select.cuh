@@ -37,6 +37,11 @@ __host__ __device__ inline size_t sel_smem_bytes(int max_blocks) {
   return 4 * nbp + 6 * 4 * W + 4 * 256 + 4 * 33 + 4 * 8 + 8 * kSmallSel + 16;
 }
 
+// Offset of the score kernel's per-chunk values after the selection scratch (16-byte aligned).
+__host__ __device__ inline size_t score_su_offset(int max_blocks) {
+  return (sel_smem_bytes(max_blocks) + 15) & ~size_t(15);
+}
+
 __device__ inline SelSmem sel_smem_carve(uint8_t* base, int max_blocks) {
   const int nbp = ((max_blocks + 31) / 32) * 32;
   const int W = nbp / 32;
@@ -385,6 +390,23 @@ __device__ int sel_topm(const SelSmem& S, const uint32_t* cand, uint32_t* out, i
     }
   }
   return m;
+}
+
+// dst[0..W) = the bits of src[0..W) whose blocks are resident in HBM (block table entry >= 0);
+// without host pools (bt NULL) every block is. Table entries are read one per thread, all of
+// a pass in flight together, and each warp assembles one word with a ballot.
+// All threads must call it; blockDim.x a multiple of 32.
+__device__ void resident_bits(const uint32_t* src, uint32_t* dst, const int32_t* bt, int W) {
+  const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  for (int j0 = 0; j0 < W * 32; j0 += nth) {
+    const int j = j0 + tid;
+    const bool in = j < W * 32 && ((src[j >> 5] >> (j & 31)) & 1u);
+    const bool keep = in && (!bt || __ldcg(bt + j) >= 0);
+    const uint32_t bw = __ballot_sync(0xffffffffu, keep);
+    const int w = (j0 >> 5) + warp;
+    if (lane == 0 && w < W) dst[w] = bw;
+  }
+  __syncthreads();
 }
 
 // Writes the set bits of mask[0..W) in ascending order to dst[rank]; returns |mask|.

@@ -86,9 +86,14 @@ def test_split_count_invariance(split):
     assert d <= 1e-6 * max(1.0, np.abs(outs[0]).max()), d
 
 
-def test_fused_equals_separate_bitwise():
+@pytest.mark.parametrize("name", ["offload_small", "llama_small"])
+def test_fused_equals_separate(name):
+    """The fused step and the separate calls select the same blocks and make the same misses,
+    bit for bit, and give the same outputs up to fp32 summation order: the fused step attends a
+    group's query-agnostic blocks first (they are published before the query-aware half),
+    the separate calls attend S(t) in ascending order."""
     import gpu_harness as H
-    c = case("offload_small")
+    c = case(name)
     res = []
     for mode in ("fused", "separate"):
         cache = H.setup(c.cfg, c.inputs)
@@ -98,6 +103,6 @@ def test_fused_equals_separate_bitwise():
             H.run_step(cache, c.cfg, c.inputs, rec, t, io, mode)
             outs.append((io.sel.cpu().numpy().copy(), io.out.cpu().numpy().copy(), io.miss.cpu().numpy().copy()))
         res.append(outs)
-    for a, b in zip(*res):
-        for x, y in zip(a, b):
-            assert np.array_equal(x, y)
+    for (sa, oa, ma), (sb, ob, mb) in zip(*res):
+        assert np.array_equal(sa, sb) and np.array_equal(ma, mb)
+        np.testing.assert_allclose(oa, ob, rtol=1e-5, atol=1e-6)
