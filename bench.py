@@ -285,6 +285,7 @@ def measure_gpu(args, cfg, rank, world, local):
                           cfg.max_blocks, slots=cfg.n_slots, n_score_rows=cfg.rows, scale=cfg.scale, score_mode=cfg.score_mode,
                           stop_tau=cfg.stop_tau, kc_bf16=cfg.kc_bf16)
     cache = nosa.NosaCache(cc, offload=cfg.offload)
+    n_kernels = nosa.step_launches(cc, cache.state)  # kernels per nosa_step
     pk = torch.from_numpy(inp.pool_k.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)
     pv = torch.from_numpy(inp.pool_v.reshape(NG, cfg.max_blocks, cfg.block, cfg.d)).view(torch.int16)
     resident = None
@@ -613,13 +614,14 @@ def measure_gpu(args, cfg, rank, world, local):
         "bytes_per_step": float(np.mean(step_b)),
         "kernel_us": {"score_select": 1e3 * float(np.mean(k_score)),
                       "gather": 1e3 * float(np.mean(k_gather)), "attention": 1e3 * attn_ms},
+        "step_kernels": n_kernels,
         "roofline": roof,
         "step0_us": 1e3 * step0_ms,
         "e2e": {"value": q_per_step / (e2e_ms / 1e3), "unit": "queries/s", "steps": n_e2e,
                 "overlap": "inputs of step i+1 and outputs of step i-1 copied during step i",
                 "l2": "not flushed: every step reads more than L2 holds",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * (3 if cfg.offload else 2),
+        "gpu_launches": args.steps * n_kernels,
         "clocks": clocks,
     }
     if pcie is not None:
@@ -767,7 +769,7 @@ def summarize(name: str, line: dict) -> dict:
          "hbm_gbs": line["hbm_gbs"], "hbm_frac": line["hbm_frac"], "bytes_per_step": line["bytes_per_step"],
          "kernel_us": line["kernel_us"], "roofline_frac": line["roofline"]["frac"],
          "roofline_kernel": line["roofline"]["kernel"], "step0_us": line["step0_us"],
-         "launch": line["launch"], "clocks": line["clocks"]}
+         "launch": line["launch"], "clocks": line["clocks"], "step_kernels": line["step_kernels"]}
     for k in ("pcie", "early_stop"):
         if k in line:
             e[k] = line[k]

@@ -218,15 +218,24 @@ nosa_status nosa_decode_attn(const nosa_config* cfg, const nosa_state* st, const
                              void* stream);
 
 /*
- * One whole decode step: append -> score -> select -> gather -> attention, in two
- * kernels (three with host pools). score_rows NULL = score with q (requires
- * n_score_rows == G). events: NULL, or 4 cudaEvent_t recorded on the stream before
- * the first kernel and after each of score/select, gather and attention (profiling).
+ * One whole decode step: append -> score -> select -> gather -> attention, in two kernels
+ * (three with host pools; nosa_step_launches reports the count). score_rows NULL = score
+ * with q (requires n_score_rows == G). events: NULL, or 4 cudaEvent_t recorded on the stream
+ * before the first kernel and after each of score/select, gather and attention (profiling).
  */
 nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16_t* q,
                       const uint16_t* score_rows, const uint16_t* k_new, const uint16_t* v_new,
                       const float* evict_scores, int32_t* sel, float* out, int32_t* miss_count,
                       void* workspace, size_t ws_bytes, void* stream, void* const* events);
+
+/*
+ * How many kernels one nosa_step launches for this configuration and state: 2 (score +
+ * selection, attention) or 3 with host pools (score + selection, page copies, attention).
+ * Launches nothing; the state is checked as nosa_step checks it (host pools: one
+ * cudaPointerGetAttributes each). kernels: host int32, written on success. Errors:
+ * NOSA_EINVAL for a bad configuration or state, or a NULL kernels.
+ */
+nosa_status nosa_step_launches(const nosa_config* cfg, const nosa_state* st, int32_t* kernels);
 
 /*
  * Lookahead decoding (SparDA, gist.science/de/paper/2606.04511, section 2: "Trainierbare

@@ -31,7 +31,8 @@ ERR_BLOCK_TABLE, ERR_SEL, ERR_NO_VICTIM, ERR_TIMEOUT, ERR_FULL, ERR_INIT = 1, 2,
 EXPORTS = ("nosa_state_sizes", "nosa_workspace_size", "nosa_workspace_init", "nosa_state_init",
            "nosa_append", "nosa_score_blocks", "nosa_select", "nosa_gather", "nosa_decode_attn",
            "nosa_step", "nosa_check_device", "nosa_status_string", "nosa_last_error",
-           "nosa_decode_attn_noalloc", "nosa_uva_read_probe", "nosa_plan_ahead", "nosa_prefetch", "nosa_attend", "nosa_stop_counts")
+           "nosa_decode_attn_noalloc", "nosa_uva_read_probe", "nosa_plan_ahead", "nosa_prefetch", "nosa_attend", "nosa_stop_counts",
+           "nosa_step_launches")
 
 
 NOSA_SCORE_WINDOW, NOSA_SCORE_SOFTMAX = 1, 2
@@ -97,6 +98,7 @@ def load(path: Optional[str] = None):
         "nosa_prefetch": [cfgp, stp, vp, sz, vp],
         "nosa_stop_counts": [cfgp, vp, sz, vp, vp],
         "nosa_attend": [cfgp, stp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "nosa_step_launches": [cfgp, stp, ctypes.POINTER(ctypes.c_int32)],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -236,6 +238,13 @@ def attend(cfg, st, q, k_new, v_new, sel, out, ws, ws_bytes, stream=None):
 def stop_counts(cfg, ws, ws_bytes, used, stream=None):
     """Blocks each query head visited in the last early-stop step ([B*Hq] int32, device)."""
     _check(load().nosa_stop_counts(ctypes.byref(cfg), _ptr(ws), ws_bytes, _ptr(used), _stream(stream)))
+
+
+def step_launches(cfg, st) -> int:
+    """Kernels nosa_step launches without events (1: the fused persistent step kernel)."""
+    n = ctypes.c_int32()
+    _check(load().nosa_step_launches(ctypes.byref(cfg), ctypes.byref(st), ctypes.byref(n)))
+    return n.value
 
 
 def check_device(st, stream=None):

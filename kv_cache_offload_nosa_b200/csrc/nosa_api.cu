@@ -738,6 +738,16 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   return rec(3);
 }
 
+nosa_status nosa_step_launches(const nosa_config* cfg, const nosa_state* st, int32_t* kernels) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  const nosa_config& c = *cfg;
+  if ((r = check_state(c, st)) != NOSA_OK) return r;
+  NOSA_CHECK(kernels, "kernels is NULL");
+  *kernels = has_host(st) ? 3 : 2;  // score + selection, [page copies,] attention
+  return NOSA_OK;
+}
+
 nosa_status nosa_plan_ahead(const nosa_config* cfg, const nosa_state* st, const uint16_t* score_rows,
                             const float* evict, int32_t* sel, int32_t* miss_count, void* ws,
                             size_t ws_bytes, void* stream) {

@@ -187,3 +187,19 @@ def test_workspace_one_byte_short_is_refused_before_any_cuda_call(lib):
     assert rc == nosa.NOSA_ENOMEM
     msg = lib.nosa_last_error().decode()
     assert str(need) in msg and str(need - 1) in msg, msg
+
+
+def test_step_launch_count_on_host(lib):
+    """nosa_step_launches answers from the configuration and state alone (no GPU: the
+    addresses are never dereferenced): every block in HBM -> 2 kernels (score + selection,
+    attention); a NULL output or a bad configuration is refused."""
+    c = cfg()
+    fake = [0x10000 * (i + 1) for i in range(12)]
+    st = nosa.nosa_state(*fake[:9], None, None, fake[9])
+    assert nosa.step_launches(c, st) == 2
+    n = ctypes.c_int32(-1)
+    assert lib.nosa_step_launches(ctypes.byref(c), ctypes.byref(st), None) == nosa.NOSA_EINVAL
+    bad = cfg()
+    bad.k_q = bad.k_e = 0
+    assert lib.nosa_step_launches(ctypes.byref(bad), ctypes.byref(st), ctypes.byref(n)) == nosa.NOSA_EINVAL
+    assert n.value == -1
