@@ -401,7 +401,7 @@ nosa_status launch_attn_stop_t(const nosa_config& c, AttnArgs a, StopArgs x, con
   using SS = StopShape<D, BS>;
   // one CTA per group, one per SM: spend the shared memory on stages
   const int G = c.Hq / c.Hkv;
-  int stages = (int)((200 * 1024 - SS::extra_bytes(G)) / SH::STAGE);
+  int stages = (int)((227 * 1024 - 1024 - SS::extra_bytes(G)) / SH::STAGE);
   stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
   const size_t smem = SS::smem_bytes(stages, G);
   auto k = attn_stop_kernel<D, BS>;
@@ -485,7 +485,7 @@ nosa_status launch_attn(const nosa_config& c, const nosa_state* st, const uint16
     a.e_flag = ws_at<uint32_t>(ws, w.e_flag);
   }
   if (c.stop_tau > 0.f) {
-    // early stop: one CTA per group, after the whole previous grid (no per-group flags)
+    // early stop: one CTA per group, each waiting for its own group's flag (or the whole grid)
     StopArgs x;
     x.scores = ws_at<float>(ws, w.scores);
     x.tau = c.stop_tau;
@@ -720,10 +720,11 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   // (which themselves start on the group's published plan) have landed. With events each
   // kernel waits for the previous one as a whole, so that the events time kernels alone.
   const WsLayout w = ws_layout(c);
-  // early stop waits for the previous grid as a whole: no per-group flags then
-  const bool flags = !events && !(c.stop_tau > 0.f);
+  const bool flags = !events;
+  // early stop ranks the whole selection before its first block: no early Gamma_e there
+  const bool early = flags && kEarlyGammaE && !(c.stop_tau > 0.f);
   a.sel_flag = flags ? ws_at<uint32_t>(ws, w.sel_flag) : nullptr;
-  if (flags && kEarlyGammaE) {
+  if (early) {
     // the query-agnostic blocks of a group are attended as soon as they are chosen
     a.att_list = ws_at<int32_t>(ws, w.att_list);
     a.e_flag = ws_at<uint32_t>(ws, w.e_flag);
@@ -734,7 +735,7 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   if ((r = rec(1)) != NOSA_OK) return r;
   if (has_host(st) && (r = launch_copy(c, st, ws, s, flags)) != NOSA_OK) return r;
   if ((r = rec(2)) != NOSA_OK) return r;
-  if ((r = launch_attn(c, st, q, sel, out, ws, s, ready, true, flags && kEarlyGammaE)) != NOSA_OK) return r;
+  if ((r = launch_attn(c, st, q, sel, out, ws, s, ready, true, early)) != NOSA_OK) return r;
   return rec(3);
 }
 

@@ -42,10 +42,11 @@ template <int D, int BS>
 struct StopShape {
   using SH = AttnShape<D, BS>;
   static constexpr int NC = SH::NC;
-  // after the stages: barriers and task infos (as attn_kernel), then the order, the ranked
-  // entries and their pages, the per-warp exchange and the final merge
+  // after the stages: barriers and task infos (as attn_kernel), then the order, the selected
+  // entries with their scores and pages, the pages in order, the per-warp exchange and the
+  // final merge
   static size_t extra_bytes(int G) {
-    return 2 * kMaxStages * 8 + kMaxStages * sizeof(TaskInfo) + 4 * (size_t)kStopMaxK * 4 +
+    return 2 * kMaxStages * 8 + kMaxStages * sizeof(TaskInfo) + 5 * (size_t)kStopMaxK * 4 +
            (size_t)NC * 8 * 3 * 4 + (size_t)NC * G * (D + 2) * 4 + 64;
   }
   static size_t smem_bytes(int stages, int G) { return 1024 + (size_t)stages * SH::STAGE + extra_bytes(G); }
@@ -68,7 +69,8 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
   int* order = reinterpret_cast<int*>(info + kMaxStages);  // block at each visiting position
   int* ent = order + kStopMaxK;                            // selected block of each entry, or -1
   float* esc = reinterpret_cast<float*>(ent + kStopMaxK);  // its score
-  int* pages = reinterpret_cast<int*>(esc + kStopMaxK);    // page of each visiting position
+  int* epg = reinterpret_cast<int*>(esc + kStopMaxK);      // its page
+  int* pages = epg + kStopMaxK;                            // page of each visiting position
   float* xch = reinterpret_cast<float*>(pages + kStopMaxK);  // [NC][8][3] (max, mass, gain)
   float* mrg = xch + NC * 8 * 3;                             // [NC][G][D+2] final merge
   volatile int* s_all_stopped = reinterpret_cast<volatile int*>(mrg + (size_t)NC * a.G * (D + 2));
@@ -87,20 +89,39 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
     tma_prefetch_desc(&tmk);
     tma_prefetch_desc(&tmv);
   }
-  // sel, the block scores, seq_len and the block table come from the previous kernels
-  griddep_wait();
+  // sel, the block scores, seq_len and the block table come from the previous kernels: wait
+  // for that whole grid, or (flags) for this group's flag, which this CTA alone waits on
+  const bool flags = a.sel_flag != nullptr;
+  if (!flags) griddep_wait();
   const unsigned long long deadline = globaltimer() + a.wait_ns;
+  if (flags && tid == 0) {
+    if (!wait_flag(a.sel_flag + (size_t)gi * kFlagStride, deadline)) set_err(a.err, NOSA_ERR_TIMEOUT);
+    a.sel_flag[(size_t)gi * kFlagStride] = 0u;
+  }
+  __syncthreads();
   const int L = __ldcg(a.seq_len + gi);
   const int N = (L + BS - 1) / BS;
-  // visiting order: selected blocks by decreasing score, ties to the lower index
+  // each selected block with its score and page (independent loads: one round trip)
   for (int w = tid; w < a.k; w += blockDim.x) {
     const int j = __ldcg(a.sel + (size_t)gi * a.k + w);
     if (j >= N) set_err(a.err, NOSA_ERR_SEL);
     const bool ok = j >= 0 && j < N;
+    float sj = 0.f;
+    int page = -1;
+    if (ok) {
+      sj = __ldcg(x.scores + (size_t)gi * a.max_blocks + j);
+      page = __ldcg(a.block_table + (size_t)gi * a.max_blocks + j);
+      if (page < 0 || page >= a.total_pages) {
+        set_err(a.err, NOSA_ERR_BLOCK_TABLE);
+        page = -1;
+      }
+    }
     ent[w] = ok ? j : -1;
-    esc[w] = ok ? __ldcg(x.scores + (size_t)gi * a.max_blocks + j) : 0.f;
+    esc[w] = sj;
+    epg[w] = page;
   }
   __syncthreads();
+  // visiting order: selected blocks by decreasing score, ties to the lower index
   for (int w = tid; w < a.k; w += blockDim.x) {
     const int j = ent[w];
     if (j < 0) continue;
@@ -111,18 +132,10 @@ __global__ void __launch_bounds__(AttnShape<D, BS>::THREADS, 1)
       rank += (j2 >= 0) && (esc[w2] > sj || (esc[w2] == sj && j2 < j));
     }
     order[rank] = j;
+    pages[rank] = epg[w];
   }
   int nvis = 0;  // selected blocks of the group
   for (int w = 0; w < a.k; ++w) nvis += (ent[w] >= 0);
-  __syncthreads();
-  for (int p = tid; p < nvis; p += blockDim.x) {
-    int page = __ldcg(a.block_table + (size_t)gi * a.max_blocks + order[p]);
-    if (page < 0 || page >= a.total_pages) {
-      set_err(a.err, NOSA_ERR_BLOCK_TABLE);
-      page = -1;
-    }
-    pages[p] = page;
-  }
   __syncthreads();
 
   if (warp == NC) {
