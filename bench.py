@@ -575,7 +575,8 @@ def measure_gpu(args, cfg, rank, world, local):
     achieved = float(np.mean(attn_b)) / (attn_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "traffic": attn_traffic(cfg.B) if cfg.name == "llama" else None,
-            "kernel": "attn_kernel", "peak_kind": peak_kind, "bytes_per_launch": float(np.mean(attn_b))}
+            "kernel": "attn_stop_kernel" if cfg.stop_tau > 0 else "attn_kernel", "peak_kind": peak_kind,
+            "bytes_per_launch": float(np.mean(attn_b))}
     pcie = None
     if cfg.offload:
         # the step is bound by the slower of its HBM bytes at the HBM peak and its PCIe bytes
