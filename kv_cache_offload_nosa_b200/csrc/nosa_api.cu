@@ -207,7 +207,7 @@ void set_ws(StepArgs& a, const nosa_config& c, void* ws) {
 // Score CTAs of 256 sub-blocks: about three waves on the Llama-shaped layer, each CTA short
 // enough that an SM's CTAs finish at staggered times. (Larger chunks, one wave of about two CTAs
 // per SM, streamed slower: fewer loads in flight.)
-constexpr int kScoreChunk = 256;
+constexpr int kScoreChunk = 384;
 // Shared-memory carveout (percent) of the score kernel, or -1 for the driver's choice, and the
 // attention's shared memory for tile stages (its carveout is the largest shared split).
 constexpr int kStepCarveout = -1;
@@ -215,9 +215,14 @@ constexpr int kAttnStageBudget = 110 * 1024;
 // The fused step publishes each group's query-agnostic blocks ahead of the rest of its selection.
 constexpr bool kEarlyGammaE = true;
 
+// Sub-blocks per score CTA: the fewest chunks of at most kScoreChunk that cover max_sub, made
+// equal (rounded up to kChunkAlign). max_sub is T/s plus one block's sub-blocks, so a fixed
+// chunk would leave every group a last CTA of a few rows.
 nosa_status score_chunk(const nosa_config& c, int* chunk) {
-  (void)c;
-  *chunk = kScoreChunk;
+  const int ms = max_sub(c);
+  const int C = (ms + kScoreChunk - 1) / kScoreChunk;
+  const int even = (ms + C - 1) / C;
+  *chunk = (even + kChunkAlign - 1) / kChunkAlign * kChunkAlign;
   return NOSA_OK;
 }
 
