@@ -217,10 +217,18 @@ constexpr bool kEarlyGammaE = true;
 
 // Sub-blocks per score CTA: the fewest chunks of at most kScoreChunk that cover max_sub, made
 // equal (rounded up to kChunkAlign). max_sub is T/s plus one block's sub-blocks, so a fixed
-// chunk would leave every group a last CTA of a few rows.
+// chunk would leave every group a last CTA of a few rows. Small batches take more, smaller
+// chunks (down to kChunkAlign), so that the grid still fills the SMs about once.
 nosa_status score_chunk(const nosa_config& c, int* chunk) {
   const int ms = max_sub(c);
-  const int C = (ms + kScoreChunk - 1) / kScoreChunk;
+  int C = (ms + kScoreChunk - 1) / kScoreChunk;
+  int dev = 0, sms = 0;
+  NOSA_CUDA(cudaGetDevice(&dev));
+  NOSA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const long long ng = n_groups(c);
+  const int want = (int)((3LL * sms + ng - 1) / ng);  // three score CTAs per SM
+  const int cmax = (ms + kChunkAlign - 1) / kChunkAlign;
+  if (C < want) C = want < cmax ? want : cmax;
   const int even = (ms + C - 1) / C;
   *chunk = (even + kChunkAlign - 1) / kChunkAlign * kChunkAlign;
   return NOSA_OK;
