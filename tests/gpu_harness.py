@@ -71,6 +71,13 @@ def run_step(cache, cfg, inputs, rec, t, io: StepIO, mode: str = "fused"):
     ev = dev(inputs.evict[t])
     if mode == "fused":
         cache.step(q, kn, vn, ev, io.sel, io.out, io.miss, score_rows=rows)
+    elif mode == "events":
+        # the profiling form of the step: events between its kernels, each kernel waiting for
+        # the previous grid as a whole instead of per-group flags
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        for e in evs:
+            e.record()  # torch creates the CUDA events when first recorded
+        cache.step(q, kn, vn, ev, io.sel, io.out, io.miss, score_rows=rows, events=evs)
     elif mode == "lookahead":
         # SparDA order on one stream: select and plan from the forecast row, copy, then
         # append and attend

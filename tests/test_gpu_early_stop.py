@@ -27,6 +27,17 @@ def test_early_stop_parity(name):
     assert mx <= H.ATOL and rl2 <= H.RTOL_L2
 
 
+@pytest.mark.parametrize("name", ["tiny_stop", "ragged_stop", "llama_small_stop"])
+def test_early_stop_parity_with_events(name):
+    """The same with events between the kernels: the stop kernel waits for the whole score
+    grid (and, with host pools, the grid-wide page copy) instead of its group's flag."""
+    _need_gpu()
+    import gpu_harness as H
+    case = O.run_case(CS[name])
+    _, (mx, rl2) = H.run_and_compare(case, mode="events")
+    assert mx <= H.ATOL and rl2 <= H.RTOL_L2
+
+
 def test_early_stop_refused_outside_the_step():
     _need_gpu()
     import gpu_harness as H

@@ -46,6 +46,15 @@ def test_step_parity_separate_calls(name):
     H.run_and_compare(case(name), mode="separate")
 
 
+@pytest.mark.parametrize("name", ["tiny", "offload_small", "ragged_offload", "llama_small", "g8"])
+def test_step_parity_with_events(name):
+    """nosa_step given events (the form bench.py times kernel by kernel): the kernels chain by
+    whole grids instead of per-group flags, and host pools go through the grid-wide copy kernel.
+    Same selections, state and outputs as the oracle."""
+    import gpu_harness as H
+    H.run_and_compare(case(name), mode="events")
+
+
 @pytest.mark.parametrize("name", ["tiny", "ragged", "bs128_d64", "g8"])
 def test_block_scores_vs_oracle(name):
     import gpu_harness as H
