@@ -238,6 +238,34 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
 nosa_status nosa_step_launches(const nosa_config* cfg, const nosa_state* st, int32_t* kernels);
 
 /*
+ * Launch geometry of the step's kernels for this configuration on a GPU with `sms` SMs on which
+ * `attn_ctas_per_sm` attention CTAs are resident at once (two on a B200 with 64-token blocks and
+ * d = 128), as nosa_step (given no events) chooses it:
+ *   score_chunk        sub-blocks per score CTA: the fewest equal chunks of at most 384 that
+ *                      cover the group's sub-blocks, rounded up to 64, and for small batches at
+ *                      least about three score CTAs per SM in all (chunks down to 64);
+ *   score_ctas         score CTAs (groups x chunks per group);
+ *   attn_tasks_per_cta (group, block) tasks per attention CTA: attn_split when set; with host
+ *                      pools the smallest width the 16 partial slots per group allow; otherwise a
+ *                      divisor of k near one CTA per resident slot, or one CTA per group when a
+ *                      group's selected K and V pages total at most 512 KB and the groups number
+ *                      between a quarter of the SMs and one wave; with early stop one CTA per
+ *                      group;
+ *   attn_ctas          attention CTAs.
+ * host_pools: nonzero for a state with host pools. No CUDA call. Errors: NOSA_EINVAL for a bad
+ * configuration, sms or attn_ctas_per_sm < 1, or a NULL out.
+ */
+typedef struct nosa_geometry {
+  int32_t score_chunk;
+  int32_t score_ctas;
+  int32_t attn_tasks_per_cta;
+  int32_t attn_ctas;
+} nosa_geometry;
+
+nosa_status nosa_step_geometry(const nosa_config* cfg, int32_t host_pools, int32_t sms,
+                               int32_t attn_ctas_per_sm, nosa_geometry* out);
+
+/*
  * Lookahead decoding (SparDA, gist.science/de/paper/2606.04511, section 2: "Trainierbare
  * Lookahead Sparse-Selektion", "Asynchrones Prefetching mit persistentem UVA-Kernel"): the
  * blocks a step attends are chosen from a forecast row before the step's query exists, so

@@ -32,7 +32,7 @@ EXPORTS = ("nosa_state_sizes", "nosa_workspace_size", "nosa_workspace_init", "no
            "nosa_append", "nosa_score_blocks", "nosa_select", "nosa_gather", "nosa_decode_attn",
            "nosa_step", "nosa_check_device", "nosa_status_string", "nosa_last_error",
            "nosa_decode_attn_noalloc", "nosa_uva_read_probe", "nosa_plan_ahead", "nosa_prefetch", "nosa_attend", "nosa_stop_counts",
-           "nosa_step_launches")
+           "nosa_step_launches", "nosa_step_geometry")
 
 
 NOSA_SCORE_WINDOW, NOSA_SCORE_SOFTMAX = 1, 2
@@ -99,6 +99,7 @@ def load(path: Optional[str] = None):
         "nosa_stop_counts": [cfgp, vp, sz, vp, vp],
         "nosa_attend": [cfgp, stp, vp, vp, vp, vp, vp, vp, sz, vp],
         "nosa_step_launches": [cfgp, stp, ctypes.POINTER(ctypes.c_int32)],
+        "nosa_step_geometry": [cfgp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -245,6 +246,18 @@ def step_launches(cfg, st) -> int:
     n = ctypes.c_int32()
     _check(load().nosa_step_launches(ctypes.byref(cfg), ctypes.byref(st), ctypes.byref(n)))
     return n.value
+
+
+class nosa_geometry(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("score_chunk", "score_ctas", "attn_tasks_per_cta", "attn_ctas")]
+
+
+def step_geometry(cfg, host_pools: bool, sms: int, attn_ctas_per_sm: int) -> dict:
+    """Launch geometry nosa_step chooses on a GPU with `sms` SMs (no CUDA call)."""
+    g = nosa_geometry()
+    _check(load().nosa_step_geometry(ctypes.byref(cfg), int(bool(host_pools)), sms, attn_ctas_per_sm,
+                                     ctypes.byref(g)))
+    return {n: getattr(g, n) for n, _ in nosa_geometry._fields_}
 
 
 def check_device(st, stream=None):

@@ -219,18 +219,22 @@ constexpr bool kEarlyGammaE = true;
 // equal (rounded up to kChunkAlign). max_sub is T/s plus one block's sub-blocks, so a fixed
 // chunk would leave every group a last CTA of a few rows. Small batches take more, smaller
 // chunks (down to kChunkAlign), so that the grid still fills the SMs about once.
-nosa_status score_chunk(const nosa_config& c, int* chunk) {
+int score_chunk_for(const nosa_config& c, int sms) {
   const int ms = max_sub(c);
   int C = (ms + kScoreChunk - 1) / kScoreChunk;
-  int dev = 0, sms = 0;
-  NOSA_CUDA(cudaGetDevice(&dev));
-  NOSA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const long long ng = n_groups(c);
   const int want = (int)((3LL * sms + ng - 1) / ng);  // three score CTAs per SM
   const int cmax = (ms + kChunkAlign - 1) / kChunkAlign;
   if (C < want) C = want < cmax ? want : cmax;
   const int even = (ms + C - 1) / C;
-  *chunk = (even + kChunkAlign - 1) / kChunkAlign * kChunkAlign;
+  return (even + kChunkAlign - 1) / kChunkAlign * kChunkAlign;
+}
+
+nosa_status score_chunk(const nosa_config& c, int* chunk) {
+  int dev = 0, sms = 0;
+  NOSA_CUDA(cudaGetDevice(&dev));
+  NOSA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  *chunk = score_chunk_for(c, sms);
   return NOSA_OK;
 }
 
@@ -350,6 +354,39 @@ nosa_status make_pool_map(CUtensorMap* m, const nosa_config& c, void* pool) {
   return NOSA_OK;
 }
 
+// Tasks ((group, block) pairs) per attention CTA. split > 0: the caller's width; finest: the
+// smallest width the partial slots allow; otherwise the automatic rule below. target = the
+// resident attention CTAs (SMs x CTAs per SM), stage = bytes of one block's K and V pages.
+int attn_split_for(int split, int k, int total, long long target, int sms, int stage, bool finest) {
+  const int wmin = (k + kPartialSlots - 2) / (kPartialSlots - 1);
+  int W = split;
+  if (W <= 0 && finest) W = wmin;
+  if (W <= 0) {
+    // Prefer a divisor of k: every CTA then holds one segment of one group and never flushes
+    // in mid-stream. Aim at about one CTA per resident slot: a single wave pays each CTA's
+    // start (flag, selection, first tiles) and flush once per slot (Llama-shaped layer:
+    // W = 32 gives 55 us of attention against 58 us at W = 16, and a shorter step).
+    const double want = (double)total / (double)target;
+    int best = 0;
+    double best_d = 1e30;
+    for (int d = wmin; d <= k; ++d) {
+      if (k % d) continue;
+      const double dist = d > want ? d / want : want / d;
+      if (dist < best_d) { best_d = dist; best = d; }
+    }
+    W = (best > 0 && best_d <= 2.0) ? best : (int)((total + target - 1) / target);
+    // Few selected pages per group (at most 512 KB of K and V), groups enough to spread over
+    // the SMs and few enough for one wave: one CTA per group. Each group's attention then
+    // starts as soon as its selection is published and needs no merge across CTAs (sweep,
+    // T=65536, bs=64, 1 %: 51 us per step against 61 us with W = 3).
+    const long long ng = total / k;
+    if (ng <= target && 4 * ng >= sms && (long long)k * stage <= 512 * 1024) W = k;
+  }
+  if (W < wmin) W = wmin;
+  if (W < 1) W = 1;
+  return W;
+}
+
 // finest: the smallest split width the partial slots allow (used when the attention of each
 // group waits for that group's page copies: groups become ready one after another over the
 // whole PCIe transfer, so spreading each group over more CTAs shortens the last group's tail).
@@ -370,32 +407,7 @@ nosa_status launch_attn_t(const nosa_config& c, AttnArgs a, const CUtensorMap& t
   NOSA_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, SH::THREADS, smem));
   if (per_sm < 1) per_sm = 1;
   const long long target = (long long)sms * per_sm;
-  const int wmin = (a.k + kPartialSlots - 2) / (kPartialSlots - 1);
-  int W = c.attn_split;
-  if (W <= 0 && finest) W = wmin;
-  if (W <= 0) {
-    // Prefer a divisor of k: every CTA then holds one segment of one group and never flushes
-    // in mid-stream. Aim at about one CTA per resident slot: a single wave pays each CTA's
-    // start (flag, selection, first tiles) and flush once per slot (Llama-shaped layer:
-    // W = 32 gives 55 us of attention against 58 us at W = 16, and a shorter step).
-    const double want = (double)a.total / (double)target;
-    int best = 0;
-    double best_d = 1e30;
-    for (int d = wmin; d <= a.k; ++d) {
-      if (a.k % d) continue;
-      const double dist = d > want ? d / want : want / d;
-      if (dist < best_d) { best_d = dist; best = d; }
-    }
-    W = (best > 0 && best_d <= 2.0) ? best : (int)((a.total + target - 1) / target);
-    // Few selected pages per group (at most 512 KB of K and V), groups enough to spread over
-    // the SMs and few enough for one wave: one CTA per group. Each group's attention then
-    // starts as soon as its selection is published and needs no merge across CTAs (sweep,
-    // T=65536, bs=64, 1 %: 51 us per step against 61 us with W = 3).
-    const long long ng = a.total / a.k;
-    if (ng <= target && 4 * ng >= sms && (long long)a.k * SH::STAGE <= 512 * 1024) W = a.k;
-  }
-  if (W < wmin) W = wmin;
-  if (W < 1) W = 1;
+  const int W = attn_split_for(c.attn_split, a.k, a.total, target, sms, SH::STAGE, finest);
   a.W = W;
   a.stages = stages;
   const int grid = (a.total + W - 1) / W;
@@ -756,6 +768,32 @@ nosa_status nosa_step(const nosa_config* cfg, const nosa_state* st, const uint16
   if ((r = rec(2)) != NOSA_OK) return r;
   if ((r = launch_attn(c, st, q, sel, out, ws, s, ready, true, early)) != NOSA_OK) return r;
   return rec(3);
+}
+
+nosa_status nosa_step_geometry(const nosa_config* cfg, int32_t host_pools, int32_t sms,
+                               int32_t attn_ctas_per_sm, nosa_geometry* out) {
+  nosa_status r = check_cfg(cfg);
+  if (r != NOSA_OK) return r;
+  NOSA_CHECK(out, "out is NULL");
+  NOSA_CHECK(sms >= 1 && attn_ctas_per_sm >= 1, "sms (%d) and attn_ctas_per_sm (%d) must be >= 1", sms,
+             attn_ctas_per_sm);
+  const nosa_config& c = *cfg;
+  const int chunk = score_chunk_for(c, sms);
+  out->score_chunk = chunk;
+  out->score_ctas = n_groups(c) * ((max_sub(c) + chunk - 1) / chunk);
+  const int k = kk(c), total = n_groups(c) * k;
+  if (c.stop_tau > 0.f) {
+    // early stop: one CTA per group visits its blocks in order
+    out->attn_tasks_per_cta = k;
+    out->attn_ctas = n_groups(c);
+    return NOSA_OK;
+  }
+  // K and V pages of one block: 2 x bs x d bf16 values
+  const int W = attn_split_for(c.attn_split, k, total, (long long)sms * attn_ctas_per_sm, sms,
+                               4 * c.block_size * c.d, host_pools != 0);
+  out->attn_tasks_per_cta = W;
+  out->attn_ctas = (total + W - 1) / W;
+  return NOSA_OK;
 }
 
 nosa_status nosa_step_launches(const nosa_config* cfg, const nosa_state* st, int32_t* kernels) {

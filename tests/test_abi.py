@@ -203,3 +203,59 @@ def test_step_launch_count_on_host(lib):
     bad.k_q = bad.k_e = 0
     assert lib.nosa_step_launches(ctypes.byref(bad), ctypes.byref(st), ctypes.byref(n)) == nosa.NOSA_EINVAL
     assert n.value == -1
+
+
+def _syn_config(name, **over):
+    import nosa_synth as syn
+    c = syn.configs()[name]
+    kw = dict(slots=c.n_slots, n_score_rows=c.rows, scale=c.scale, score_mode=c.score_mode,
+              stop_tau=c.stop_tau, kc_bf16=c.kc_bf16)
+    kw.update(over)
+    return c, nosa.make_config(c.B, c.Hq, c.Hkv, c.d, c.block, c.sub_block, c.k_q, c.k_e, c.max_blocks, **kw)
+
+
+@pytest.mark.parametrize("name,host,want", [
+    # Llama-shaped: 2052 sub-blocks per group in 6 chunks of 384; k = 64 in halves (one CTA per
+    # resident slot: 296 slots, 256 CTAs)
+    ("llama", False, dict(score_chunk=384, score_ctas=128 * 6, attn_tasks_per_cta=32, attn_ctas=256)),
+    # sink: 1028 sub-blocks in 3 chunks; k = 32, 1 MB of pages per group: the divisor rule, W = 32
+    ("sink", False, dict(score_chunk=384, score_ctas=256 * 3, attn_tasks_per_cta=32, attn_ctas=256)),
+    # T = 65536, 1 %: k = 11 pages (352 KB) per group, 64 groups: one CTA per group
+    ("sweep_T65536_b64_p1", False, dict(score_chunk=384, score_ctas=64 * 11, attn_tasks_per_cta=11, attn_ctas=64)),
+    # k = 103 is prime and 3.4 MB per group: no divisor near a CTA per slot, W = ceil(6592 / 296)
+    ("sweep_T65536_b64_p10", False, dict(score_chunk=384, score_ctas=64 * 11, attn_tasks_per_cta=23, attn_ctas=287)),
+    # tiny: 2 groups, so at least ~3 score CTAs per SM in all means 5 chunks of 64 sub-blocks
+    # (260 in all); the attention keeps the smallest width the 16 partial slots allow
+    ("tiny", False, dict(score_chunk=64, score_ctas=2 * 5, attn_tasks_per_cta=2, attn_ctas=16)),
+    # offload: 8196 sub-blocks in 22 chunks; with host pools the finest split, ceil(128 / 15)
+    ("offload", True, dict(score_chunk=384, score_ctas=32 * 22, attn_tasks_per_cta=9, attn_ctas=456)),
+    # early stop: one CTA per group
+    ("llama_stop", False, dict(score_chunk=384, score_ctas=128 * 6, attn_tasks_per_cta=64, attn_ctas=128)),
+])
+def test_step_geometry(lib, name, host, want):
+    """The launch geometry nosa_step picks on a B200 (148 SMs, two attention CTAs per SM),
+    computed on the host from the configuration alone."""
+    _, cc = _syn_config(name)
+    assert nosa.step_geometry(cc, host, 148, 2) == want
+
+
+def test_step_geometry_rules(lib):
+    """An explicit split is kept; the score chunks cover every sub-block with at most 384 per
+    CTA and are multiples of 64; bad arguments are refused."""
+    c, cc = _syn_config("llama", attn_split=8)
+    g = nosa.step_geometry(cc, False, 148, 2)
+    assert g["attn_tasks_per_cta"] == 8 and g["attn_ctas"] == 128 * 64 // 8
+    import nosa_synth as syn
+    for name, s in syn.configs().items():
+        _, cfg = _syn_config(name)
+        g = nosa.step_geometry(cfg, s.offload, 148, 2)
+        ch = g["score_chunk"]
+        assert ch % 64 == 0 and 64 <= ch <= 384, (name, ch)
+        per_group = g["score_ctas"] // (s.B * s.Hkv)
+        assert (per_group - 1) * ch < s.max_sub <= per_group * ch, (name, ch, per_group)
+        W = g["attn_tasks_per_cta"]
+        assert g["attn_ctas"] == -(-s.B * s.Hkv * s.k // W), name
+        assert -(-(s.k - 1) // W) + 1 <= 16, (name, W)  # a group spans at most 16 partial slots
+    out = nosa.nosa_geometry()
+    assert lib.nosa_step_geometry(ctypes.byref(cc), 0, 0, 2, ctypes.byref(out)) == nosa.NOSA_EINVAL
+    assert lib.nosa_step_geometry(ctypes.byref(cc), 0, 148, 2, None) == nosa.NOSA_EINVAL
